@@ -1,0 +1,448 @@
+"""fp64 CPU oracle: branch attention forward / backward written from its definition.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring): the product path never
+imports this module.
+
+Source: "Online Draft Co-Training" paper pages (arXiv 2609.07108):
+  - technical-contribution and method-detail sections: each branch query is the
+    causal attention over the main sequence up to its anchor plus the
+    attention over its own (rank-local) branch keys; the two partials
+    (O_m, l_m) and (O_b, l_b) combine as l = log(e^{l_m} + e^{l_b}),
+    O = e^{l_m - l} O_m + e^{l_b - l} O_b;
+  - core-innovation section: zigzag sharding of the packed main sequence,
+    branch K/V kept with the anchor's shard, main K/V visiting every shard.
+Shapes of the three draft-branch kinds (TTT-causal, block-bidirectional,
+block-causal) follow the EAGLE-3 / DFlash / DSpark description in the
+research-background section.
+
+Conventions (the reading stated in the design notes):
+  * main tokens t = 0..N-1 packed by cu_seqlens; branch b has anchor a_b and
+    depth D_b, its tokens are branch rows cu_branch[b] .. cu_branch[b+1]-1
+    (anchor-major, depth-minor);
+  * main query r sees main keys of its own sequence at positions <= r;
+  * branch query (b, j) sees main keys of the anchor's sequence at positions
+    <= a_b (anchor inclusive) and branch keys (b, j') with j' <= j (TTT-causal,
+    block-causal) or all j' (block-bidirectional);
+  * scores S = scale * q . k, LSE in natural log with the scale included;
+  * q head h reads kv head h // (Hq / Hkv).
+Everything is computed in float64 from the exact bf16 input values.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Sequence, Tuple
+
+import numpy as np
+
+MASK_TTT_CAUSAL = 0
+MASK_BLOCK_BIDIR = 1
+MASK_BLOCK_CAUSAL = 2
+
+
+def to64(x) -> np.ndarray:
+    """bf16/fp32 torch tensor or numpy array -> float64 numpy (exact)."""
+    if isinstance(x, np.ndarray):
+        return x.astype(np.float64, copy=False)
+    import torch
+    return x.detach().to("cpu", torch.float64).numpy()
+
+
+@dataclasses.dataclass
+class Derived:
+    cu: np.ndarray          # [S+1] cu_seqlens
+    cu_branch: np.ndarray   # [n_br+1] exclusive scan of depths
+    branch_seq: np.ndarray  # [n_br] sequence of each branch's anchor
+    main_seq: np.ndarray    # [N] sequence of each main token
+    row_branch: np.ndarray  # [Nb] branch of each branch row
+    n_main: int
+    n_branch_tokens: int
+
+
+def derive(st) -> Derived:
+    cu = np.asarray(st.cu_seqlens, dtype=np.int64)
+    anchors = np.asarray(st.anchors, dtype=np.int64)
+    depths = np.asarray(st.depths, dtype=np.int64)
+    n = int(cu[-1])
+    cu_branch = np.zeros(anchors.shape[0] + 1, dtype=np.int64)
+    for b in range(anchors.shape[0]):
+        cu_branch[b + 1] = cu_branch[b] + depths[b]
+    main_seq = np.zeros(n, dtype=np.int64)
+    for s in range(cu.shape[0] - 1):
+        main_seq[cu[s]:cu[s + 1]] = s
+    branch_seq = main_seq[anchors] if anchors.shape[0] else np.zeros(0, dtype=np.int64)
+    nb = int(cu_branch[-1])
+    row_branch = np.zeros(nb, dtype=np.int64)
+    for b in range(anchors.shape[0]):
+        row_branch[cu_branch[b]:cu_branch[b + 1]] = b
+    return Derived(cu, cu_branch, branch_seq, main_seq, row_branch, n, nb)
+
+
+def visible_keys(st, dv: Derived, kind: str, row: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Visible (main key indices, branch key rows) of one query row."""
+    if kind == "main":
+        s = dv.main_seq[row]
+        return np.arange(dv.cu[s], row + 1), np.zeros(0, dtype=np.int64)
+    b = dv.row_branch[row]
+    a = int(st.anchors[b])
+    s = dv.branch_seq[b]
+    main = np.arange(dv.cu[s], a + 1)
+    if st.mask_kind == MASK_BLOCK_BIDIR:
+        loc = np.arange(dv.cu_branch[b], dv.cu_branch[b + 1])
+    else:
+        loc = np.arange(dv.cu_branch[b], row + 1)
+    return main, loc
+
+
+def dense_mask(st, dv: Derived = None) -> np.ndarray:
+    """Explicit boolean mask over main+branch tokens: rows = queries, cols = keys.
+
+    Index order on both axes: main tokens 0..N-1, then branch rows N..N+Nb-1.
+    """
+    dv = dv or derive(st)
+    n, nb = dv.n_main, dv.n_branch_tokens
+    m = np.zeros((n + nb, n + nb), dtype=bool)
+    for r in range(n):
+        mk, _ = visible_keys(st, dv, "main", r)
+        m[r, mk] = True
+    for r in range(nb):
+        mk, lk = visible_keys(st, dv, "branch", r)
+        m[n + r, mk] = True
+        m[n + r, n + lk] = True
+    return m
+
+
+def _softmax_attend(s: np.ndarray, mask: np.ndarray, v: np.ndarray):
+    """Masked softmax attention of score rows s [R, T] over values v [T, d].
+
+    Rows with no visible key return O = 0 and lse = -inf (empty partial).
+    """
+    s = np.where(mask, s, -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    empty = ~np.isfinite(m[:, 0])
+    m = np.where(np.isfinite(m), m, 0.0)
+    p = np.exp(s - m)
+    z = p.sum(axis=1, keepdims=True)
+    with np.errstate(divide="ignore"):
+        lse = (m + np.log(z))[:, 0]
+    lse[empty] = -np.inf
+    zs = np.where(z > 0, z, 1.0)
+    o = (p / zs) @ v
+    o[empty] = 0.0
+    return o, lse
+
+
+def _all_tokens(t, keys: Sequence[str]):
+    return [np.concatenate([to64(t[k + "_m"]), to64(t[k + "_b"])], axis=0) for k in keys]
+
+
+def forward_dense(st, t, mask: np.ndarray = None):
+    """Union-softmax forward over the explicit mask (small problems)."""
+    dv = derive(st)
+    mask = dense_mask(st, dv) if mask is None else mask
+    q, k, v = _all_tokens(t, ["q", "k", "v"])
+    hq, hkv = st.hq, st.hkv
+    grp = hq // hkv
+    n = dv.n_main
+    o = np.zeros_like(q)
+    lse = np.zeros((hq, q.shape[0]))
+    for h in range(hq):
+        g = h // grp
+        s = st.scale * (q[:, h, :] @ k[:, g, :].T)
+        o[:, h, :], lse[h] = _softmax_attend(s, mask, v[:, g, :])
+    return o[:n], o[n:], lse[:, :n], lse[:, n:]
+
+
+def backward_dense(st, t, mask: np.ndarray = None):
+    """Analytic gradients of sum(O * dO) over the explicit mask (small problems).
+
+    D_i = dO_i . O_i; dV = P^T dO; dP = dO V^T; dS = P (dP - D);
+    dQ = scale dS K; dK = scale dS^T Q; dK/dV summed over each GQA group.
+    """
+    dv = derive(st)
+    mask = dense_mask(st, dv) if mask is None else mask
+    q, k, v, do = _all_tokens(t, ["q", "k", "v", "do"])
+    hq, hkv = st.hq, st.hkv
+    grp = hq // hkv
+    n = dv.n_main
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dvv = np.zeros_like(v)
+    for h in range(hq):
+        g = h // grp
+        s = st.scale * (q[:, h, :] @ k[:, g, :].T)
+        o, lse = _softmax_attend(s, mask, v[:, g, :])
+        p = np.where(mask, np.exp(np.where(mask, s, 0.0) - lse[:, None]), 0.0)
+        dd = (do[:, h, :] * o).sum(axis=1)
+        dvv[:, g, :] += p.T @ do[:, h, :]
+        dp = do[:, h, :] @ v[:, g, :].T
+        ds = p * (dp - dd[:, None])
+        dq[:, h, :] = st.scale * (ds @ k[:, g, :])
+        dk[:, g, :] += st.scale * (ds.T @ q[:, h, :])
+    return dq[:n], dk[:n], dvv[:n], dq[n:], dk[n:], dvv[n:]
+
+
+def lse_merge(o_a, l_a, o_b, l_b):
+    """Online-softmax merge of two partials (paper: technical contribution).
+
+    l = log(e^{l_a} + e^{l_b}),  O = e^{l_a - l} O_a + e^{l_b - l} O_b,
+    evaluated stably as l = m + log(e^{l_a - m} + e^{l_b - m}), m = max(l_a, l_b).
+    An empty partial has l = -inf, O = 0; two empty partials give (0, -inf).
+    Shapes: o_* [..., d], l_* [...].
+    """
+    o_a = np.asarray(o_a, dtype=np.float64)
+    o_b = np.asarray(o_b, dtype=np.float64)
+    l_a = np.asarray(l_a, dtype=np.float64)
+    l_b = np.asarray(l_b, dtype=np.float64)
+    m = np.maximum(l_a, l_b)
+    both_empty = ~np.isfinite(m)
+    ms = np.where(both_empty, 0.0, m)
+    with np.errstate(divide="ignore"):
+        l = ms + np.log(np.exp(l_a - ms) + np.exp(l_b - ms))
+    l = np.where(both_empty, -np.inf, l)
+    ls = np.where(both_empty, 0.0, l)
+    wa = np.where(both_empty, 0.0, np.exp(l_a - ls))
+    wb = np.where(both_empty, 0.0, np.exp(l_b - ls))
+    o = wa[..., None] * o_a + wb[..., None] * o_b
+    return o, l
+
+
+def _partial_dense(st, t, mask, cols):
+    """Partial attention of every query over the key columns selected by `cols`."""
+    sub = mask & cols[None, :]
+    return forward_dense(st, t, mask=sub)
+
+
+def split_forward(st, t):
+    """Main-prefix partial and branch-local partial, merged by the LSE rule.
+
+    Returns (o_m, o_b, lse_m, lse_b) of the merged result plus the two partials.
+    """
+    dv = derive(st)
+    mask = dense_mask(st, dv)
+    n = dv.n_main
+    total = mask.shape[1]
+    is_main = np.arange(total) < n
+    pm = _partial_dense(st, t, mask, is_main)
+    pb = _partial_dense(st, t, mask, ~is_main)
+    # merge per token group: o [rows, H, d], lse [H, rows]
+    out = []
+    for part in range(2):  # 0 = main rows, 1 = branch rows
+        o_a, l_a = pm[part], pm[2 + part]
+        o_b, l_b = pb[part], pb[2 + part]
+        o, l = lse_merge(o_a.transpose(1, 0, 2), l_a, o_b.transpose(1, 0, 2), l_b)
+        out.append((o.transpose(1, 0, 2), l))
+    return (out[0][0], out[1][0], out[0][1], out[1][1]), pm, pb
+
+
+def zigzag_chunks(cu: np.ndarray, C: int) -> List[List[Tuple[int, int]]]:
+    """Chunk k of sequence s is [cu[s] + floor(k L / 2C), cu[s] + floor((k+1) L / 2C))."""
+    out = []
+    for s in range(cu.shape[0] - 1):
+        start, L = int(cu[s]), int(cu[s + 1] - cu[s])
+        out.append([(start + (k * L) // (2 * C), start + ((k + 1) * L) // (2 * C))
+                    for k in range(2 * C)])
+    return out
+
+
+def _shard_of_chunk(k: int, C: int) -> int:
+    return k if k < C else 2 * C - 1 - k
+
+
+def zigzag_forward(st, t, C: int):
+    """Virtual zigzag ring over C shards, merged by the LSE rule.
+
+    Shard i holds chunks i and 2C-1-i of every sequence (core-innovation
+    section: packed, load-balanced zigzag) and the branches anchored in them.
+    At ring step s shard i attends its queries to the main keys held by shard
+    (i - s) mod C under the global mask; the partials are merged in step order
+    into a running (O, l), and the rank-local branch partial is merged last.
+    """
+    dv = derive(st)
+    mask = dense_mask(st, dv)
+    n, nb = dv.n_main, dv.n_branch_tokens
+    chunks = zigzag_chunks(dv.cu, C)
+    key_shard = np.full(n + nb, -1, dtype=np.int64)
+    for s_chunks in chunks:
+        for k, (lo, hi) in enumerate(s_chunks):
+            key_shard[lo:hi] = _shard_of_chunk(k, C)
+    q_shard = key_shard.copy()
+    anchors = np.asarray(st.anchors, dtype=np.int64)
+    for r in range(nb):
+        q_shard[n + r] = key_shard[anchors[dv.row_branch[r]]]
+    hq, d = st.hq, st.head_dim
+    acc_o = np.zeros((hq, n + nb, d))
+    acc_l = np.full((hq, n + nb), -np.inf)
+    for step in range(C):
+        for i in range(C):
+            j = (i - step) % C
+            rows = q_shard == i
+            cols = key_shard == j  # branch columns are -1: never main keys of a shard
+            sub = mask & rows[:, None] & cols[None, :]
+            o_m, o_b, l_m, l_b = forward_dense(st, t, mask=sub)
+            o = np.concatenate([o_m, o_b], axis=0).transpose(1, 0, 2)
+            l = np.concatenate([l_m, l_b], axis=1)
+            acc_o, acc_l = lse_merge(acc_o, acc_l, o, l)
+    is_branch = np.arange(n + nb) >= n
+    sub = mask & is_branch[None, :]
+    o_m, o_b, l_m, l_b = forward_dense(st, t, mask=sub)
+    o = np.concatenate([o_m, o_b], axis=0).transpose(1, 0, 2)
+    l = np.concatenate([l_m, l_b], axis=1)
+    acc_o, acc_l = lse_merge(acc_o, acc_l, o, l)
+    acc_o = acc_o.transpose(1, 0, 2)
+    return acc_o[:n], acc_o[n:], acc_l[:, :n], acc_l[:, n:]
+
+
+# ---------------------------------------------------------------------------
+# Row-wise evaluation for large problems (same definition, one query at a time
+# or a batch of queries from one sequence, keys gathered per row).
+# ---------------------------------------------------------------------------
+
+def _row_sets(st, dv, main_rows, branch_rows):
+    items = []
+    for r in main_rows:
+        mk, lk = visible_keys(st, dv, "main", int(r))
+        items.append(("main", int(r), mk, lk))
+    for r in branch_rows:
+        mk, lk = visible_keys(st, dv, "branch", int(r))
+        items.append(("branch", int(r), mk, lk))
+    return items
+
+
+def rows_forward(st, t, main_rows=(), branch_rows=(), with_dq=False, heads=None):
+    """Forward (and optionally dQ) of selected query rows, each from its own key set.
+
+    Returns dict with o [R, Hq, d], lse [Hq, R] and, if with_dq, dq [R, Hq, d],
+    in the order main_rows then branch_rows.  Only q heads in `heads` (default:
+    all) are computed; the others stay zero.
+    """
+    dv = derive(st)
+    items = _row_sets(st, dv, main_rows, branch_rows)
+    hq, hkv, d = st.hq, st.hkv, st.head_dim
+    grp = hq // hkv
+    heads = list(range(hq)) if heads is None else [int(h) for h in heads]
+    R = len(items)
+    o = np.zeros((R, hq, d))
+    lse = np.zeros((hq, R))
+    dq = np.zeros((R, hq, d)) if with_dq else None
+    # A row's main keys are always a prefix [cu[s], hi] of one sequence, so
+    # rows are grouped by sequence and read views of one converted prefix.
+    by_seq: Dict[int, List[int]] = {}
+    for i, (kind, r, mk, lk) in enumerate(items):
+        by_seq.setdefault(int(dv.main_seq[mk[0]]), []).append(i)
+    groups = sorted({h // grp for h in heads})
+    for s, idx in by_seq.items():
+        lo = int(dv.cu[s])
+        hi = max(int(items[i][2][-1]) for i in idx) + 1
+        for g in groups:
+            km = to64(t["k_m"][lo:hi, g])
+            vm = to64(t["v_m"][lo:hi, g])
+            for i in idx:
+                kind, r, mk, lk = items[i]
+                assert mk[0] == lo and mk[-1] == lo + mk.size - 1
+                nm = mk.size
+                sfx = "m" if kind == "main" else "b"
+                qx = to64(t["q_" + sfx][r])
+                dox = to64(t["do_" + sfx][r]) if with_dq else None
+                kl = to64(t["k_b"][lk, g]) if lk.size else np.zeros((0, d))
+                vl = to64(t["v_b"][lk, g]) if lk.size else np.zeros((0, d))
+                for h in heads:
+                    if h // grp != g:
+                        continue
+                    sc = st.scale * np.concatenate([km[:nm] @ qx[h], kl @ qx[h]])
+                    m = sc.max()
+                    p = np.exp(sc - m)
+                    z = p.sum()
+                    lse[h, i] = m + np.log(z)
+                    p = p / z
+                    o[i, h] = p[:nm] @ vm[:nm] + p[nm:] @ vl
+                    if with_dq:
+                        dp = np.concatenate([vm[:nm] @ dox[h], vl @ dox[h]])
+                        dd = float(dox[h] @ o[i, h])
+                        ds = p * (dp - dd)
+                        dq[i, h] = st.scale * (ds[:nm] @ km[:nm] + ds[nm:] @ kl)
+    out = {"o": o, "lse": lse}
+    if with_dq:
+        out["dq"] = dq
+    return out
+
+
+def rows_backward_dq(st, t, main_rows=(), branch_rows=(), heads=None):
+    return rows_forward(st, t, main_rows, branch_rows, with_dq=True, heads=heads)
+
+
+def keys_backward(st, t, main_keys=(), branch_keys=()):
+    """dK and dV of selected key rows: every query that sees them, in full.
+
+    Returns dict with dk_m/dv_m [len(main_keys), Hkv, d] and dk_b/dv_b
+    [len(branch_keys), Hkv, d].
+    """
+    dv = derive(st)
+    n, nb = dv.n_main, dv.n_branch_tokens
+    hq, hkv, d = st.hq, st.hkv, st.head_dim
+    grp = hq // hkv
+    main_keys = [int(k) for k in main_keys]
+    branch_keys = [int(k) for k in branch_keys]
+    anchors = np.asarray(st.anchors, dtype=np.int64)
+    # queries that see any selected key
+    q_main, q_branch = set(), set()
+    for k in main_keys:
+        s = dv.main_seq[k]
+        q_main.update(range(k, int(dv.cu[s + 1])))
+        for b in np.nonzero((anchors >= k) & (dv.branch_seq == s))[0]:
+            q_branch.update(range(int(dv.cu_branch[b]), int(dv.cu_branch[b + 1])))
+    for k in branch_keys:
+        b = dv.row_branch[k]
+        q_branch.update(range(int(dv.cu_branch[b]), int(dv.cu_branch[b + 1])))
+    q_main = sorted(q_main)
+    q_branch = sorted(q_branch)
+    fw = rows_forward(st, t, q_main, q_branch)
+    items = _row_sets(st, dv, q_main, q_branch)
+    mk_pos = {k: i for i, k in enumerate(main_keys)}
+    bk_pos = {k: i for i, k in enumerate(branch_keys)}
+    dk_m = np.zeros((len(main_keys), hkv, d))
+    dv_m = np.zeros((len(main_keys), hkv, d))
+    dk_b = np.zeros((len(branch_keys), hkv, d))
+    dv_b = np.zeros((len(branch_keys), hkv, d))
+    for i, (kind, r, mk, lk) in enumerate(items):
+        sel_m = [(j, mk_pos[int(k)]) for j, k in enumerate(mk) if int(k) in mk_pos]
+        sel_b = [(j, bk_pos[int(k)]) for j, k in enumerate(lk) if int(k) in bk_pos]
+        if not sel_m and not sel_b:
+            continue
+        qx = to64(t["q_" + ("m" if kind == "main" else "b")][r])
+        dox = to64(t["do_" + ("m" if kind == "main" else "b")][r])
+        kk = np.concatenate([to64(t["k_m"][mk]), to64(t["k_b"][lk]) if lk.size
+                             else np.zeros((0, hkv, d))], axis=0)
+        vv = np.concatenate([to64(t["v_m"][mk]), to64(t["v_b"][lk]) if lk.size
+                             else np.zeros((0, hkv, d))], axis=0)
+        for h in range(hq):
+            g = h // grp
+            sc = st.scale * (kk[:, g, :] @ qx[h])
+            p = np.exp(sc - fw["lse"][h, i])
+            dp = vv[:, g, :] @ dox[h]
+            dd = float(dox[h] @ fw["o"][i, h])
+            ds = p * (dp - dd)
+            for j, pos in sel_m:
+                dv_m[pos, g] += p[j] * dox[h]
+                dk_m[pos, g] += st.scale * ds[j] * qx[h]
+            off = mk.size
+            for j, pos in sel_b:
+                dv_b[pos, g] += p[off + j] * dox[h]
+                dk_b[pos, g] += st.scale * ds[off + j] * qx[h]
+    return {"dk_m": dk_m, "dv_m": dv_m, "dk_b": dk_b, "dv_b": dv_b}
+
+
+def useful_pairs(st) -> int:
+    """Number of unmasked (query head, key) pairs, summed over all q heads."""
+    dv = derive(st)
+    total = 0
+    for r in range(dv.n_main):
+        total += r - int(dv.cu[dv.main_seq[r]]) + 1
+    anchors = np.asarray(st.anchors, dtype=np.int64)
+    for b in range(anchors.shape[0]):
+        a = int(anchors[b])
+        main = a - int(dv.cu[dv.branch_seq[b]]) + 1
+        depth = int(dv.cu_branch[b + 1] - dv.cu_branch[b])
+        for j in range(depth):
+            loc = depth if st.mask_kind == MASK_BLOCK_BIDIR else j + 1
+            total += main + loc
+    return total * st.hq
