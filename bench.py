@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Branch attention fwd+bwd benchmark (one JSON line on rank 0).
+
+Workload (default): the EAGLE-3 TTT draft layer of a Qwen3-8B-shaped target,
+20,480 packed main tokens (sequence lengths uniform in [1024, 8192], last one
+cut), a depth-3 branch at every main position (61,440 branch tokens), 32 q / 8
+kv heads, head_dim 128, bf16 N(0, 1) synthetic data.
+
+One step = the whole hot path over one batch: ba_plan (tile metadata),
+branch_attn_fwd (main causal + branch prefix + branch-local, LSE-merged) and
+branch_attn_bwd (D preprocess, dQ/dK/dV recomputing P from the merged LSE,
+dQ convert).  Metric: useful-pair TFLOP/s = 10 d x (unmasked query-head x key
+pairs) / step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun) each rank runs an independent replica of the batch
+(weak scaling: the path has no cross-GPU exchange at this layout); the step
+time is the max over ranks.  `--impl reference` times the fp64 CPU oracle on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "branch-attn fwd+bwd useful-pair TFLOP/s and % of B200 BF16 tensor peak"
+UNIT = "TFLOP/s"
+SPEC_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="ttt_20k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def rank_info():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        # median over samples taken under load (clock above idle)
+        loaded = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "speculative_draft_branch_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still
+    describes the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"source_sha:\s*([0-9a-f]+)", text)
+    if not m or not s or s.group(1) != kernel_source_sha():
+        return None
+    return float(m.group(1))
+
+
+def useful_pairs_from_plan(runner) -> int:
+    """Unmasked (query head, key) pairs from the library's per-row key intervals."""
+    iv = runner.read_plan()["row_iv"]
+    main = (iv[:, 1] - iv[:, 0] + 1).sum()
+    loc = np.maximum(iv[:, 3] - iv[:, 2] + 1, 0).sum()
+    return int(main + loc) * runner.problem.c.hq
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(st, t, rng, n_rows):
+    """A bounded sample of the workload for the fp64 oracle: n_rows main rows
+    and 3 n_rows branch rows of one sequence (fwd O, LSE and dQ, all heads)."""
+    import oracle
+    seq = int(rng.integers(0, st.n_seqs))
+    lo, hi = int(st.cu_seqlens[seq]), int(st.cu_seqlens[seq + 1])
+    mr = sorted(rng.choice(np.arange(lo, hi), size=min(n_rows, hi - lo), replace=False).tolist())
+    dv = oracle.derive(st)
+    br_all = np.nonzero(dv.branch_seq[dv.row_branch] == seq)[0] if st.n_branches else []
+    br = sorted(rng.choice(br_all, size=min(3 * n_rows, len(br_all)), replace=False).tolist()) \
+        if len(br_all) else []
+    iv = oracle.row_intervals(st)
+    rows = np.array(mr + [st.n_main + b for b in br], dtype=np.int64)
+    pairs = int(((iv[rows, 1] - iv[rows, 0] + 1) + np.maximum(iv[rows, 3] - iv[rows, 2] + 1, 0)
+                 ).sum()) * st.hq
+    return mr, br, pairs
+
+
+def time_oracle(st, t, seconds_target, seed=0, n_rows=8):
+    """Runs oracle samples until ~seconds_target elapsed; returns pairs/s etc."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    total_pairs, total_s, samples = 0, 0.0, 0
+    while samples == 0 or total_s < seconds_target:
+        mr, br, pairs = oracle_sample(st, t, rng, n_rows)
+        t0 = time.perf_counter()
+        oracle.rows_backward_dq(st, t, mr, br)
+        total_s += time.perf_counter() - t0
+        total_pairs += pairs
+        samples += 1
+    return total_pairs, total_s, samples
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def workload_config(st, pairs, name, in_bytes):
+    import workloads as wl
+    return {"workload": f"{name}: {st.n_main} packed main tokens in {st.n_seqs} sequences, "
+                        f"{st.n_branches} branches ({st.n_branch_tokens} branch tokens), "
+                        f"{st.hq} q / {st.hkv} kv heads, head_dim {st.head_dim}, "
+                        f"{wl.MASK_NAMES[st.mask_kind]} branch mask",
+            "n_main": st.n_main, "n_branch_tokens": st.n_branch_tokens, "hq": st.hq,
+            "hkv": st.hkv, "head_dim": st.head_dim, "mask": wl.MASK_NAMES[st.mask_kind],
+            "useful_pairs": pairs,
+            "l2": f"inputs larger than L2: {in_bytes / 1e9:.2f} GB of tensors read per step "
+                  f"(L2 {L2_BYTES / 2**20:.0f} MiB); no explicit flush"}
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world, _ = rank_info()
+    if rank != 0:
+        return 0
+    import torch
+    import workloads as wl
+    st = wl.structure(args.workload)
+    t = wl.tensors(st, wl.workload_seed(args.workload), "cpu")
+    flop_per_pair = 10 * st.head_dim
+    # per step: one bounded oracle sample (~1-2 s of CPU work)
+    for i in range(args.warmup):
+        time_oracle(st, t, 0.0, seed=1000 + i, n_rows=4)
+    pairs, secs, _ = 0, 0.0, 0
+    for i in range(args.steps):
+        p, s, _ = time_oracle(st, t, 0.0, seed=i, n_rows=4)
+        pairs += p
+        secs += s
+    value = pairs * flop_per_pair / secs / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(st, int(pairs / args.steps), args.workload,
+                                  sum(x.numel() * x.element_size() for x in t.values())),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "per step: 4 main rows and 12 branch rows of one random "
+                                   "sequence, all heads, fwd O/LSE + dQ (10 d per pair)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import speculative_draft_branch_b200 as ba
+    import workloads as wl
+
+    rank, world, local_rank = rank_info()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    st = wl.structure(args.workload)
+    t = wl.tensors(st, wl.workload_seed(args.workload) + 1000 * rank, dev)
+    prob = ba.Problem.from_structure(st, device=dev)
+    runner = ba.BranchAttention(prob, device=dev)
+    out = runner.alloc_outputs()
+    grads = runner.alloc_grads()
+    runner.plan()
+    if runner.plan_status() != 0:
+        raise RuntimeError("plan content checks failed")
+    pairs = useful_pairs_from_plan(runner)
+    d = st.head_dim
+    flops_step = 10 * d * pairs
+    in_bytes = sum(x.numel() * x.element_size() for x in t.values())
+    stream = torch.cuda.current_stream()
+
+    def step():
+        runner.plan()
+        runner.forward(t, out)
+        runner.backward(t, out, grads)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+
+    K = args.steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    fs, fe, bs, be = [ev() for _ in range(K)], [ev() for _ in range(K)], \
+        [ev() for _ in range(K)], [ev() for _ in range(K)]
+    e0, e1 = ev(), ev()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    launches0 = ba.ba_launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(K):
+        ba.ba_set_kernel_events(0, fs[i], fe[i])
+        ba.ba_set_kernel_events(1, bs[i], be[i])
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = ba.ba_launch_count() - launches0
+    ba.ba_set_kernel_events(0, None, None)
+    ba.ba_set_kernel_events(1, None, None)
+    clk = clocks.stop()
+    total_ms = e0.elapsed_time(e1)
+    fwd_ms = [fs[i].elapsed_time(fe[i]) for i in range(K)]
+    bwd_ms = [bs[i].elapsed_time(be[i]) for i in range(K)]
+    t_max = torch.tensor([total_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    total_ms = float(t_max.item())
+    ms_step = total_ms / K
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+
+    # plan time alone (outside the timed region)
+    p0, p1 = ev(), ev()
+    p0.record(stream)
+    for _ in range(5):
+        runner.plan()
+    p1.record(stream)
+    torch.cuda.synchronize()
+    plan_ms = p0.elapsed_time(p1) / 5
+
+    pk, pk_kind = peaks()
+    fwd_avg, bwd_avg = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    fwd_flops, bwd_flops = 4 * d * pairs, 10 * d * pairs
+    dom = "bwd" if bwd_avg >= fwd_avg else "fwd"
+    dom_ms, dom_flops = (bwd_avg, bwd_flops) if dom == "bwd" else (fwd_avg, fwd_flops)
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    peak = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
+    kernel_name = "bwd_attention" if dom == "bwd" else "fwd_attention"
+    traffic = profiled_traffic(kernel_name, args.workload)
+
+    # e2e: host buffers -> device, plan/fwd/bwd through the public API, results back
+    e2e = None
+    if not args.no_e2e:
+        host_in = {k: v.cpu().pin_memory() for k, v in t.items()}
+        idx_host = [x.cpu().pin_memory() for x in (prob.cu_seqlens, prob.branch_anchor,
+                                                      prob.branch_depth)]
+        idx_dev = [prob.cu_seqlens, prob.branch_anchor, prob.branch_depth]
+        host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                    for k, v in list(out.items()) + list(grads.items())}
+        dev_out = dict(out)
+        dev_out.update(grads)
+        h2d = sum(x.numel() * x.element_size() for x in host_in.values()) + \
+            sum(x.numel() * x.element_size() for x in idx_host)
+        d2h = sum(x.numel() * x.element_size() for x in host_out.values())
+        E = max(3, min(K, 10))
+
+        def e2e_step():
+            for k, v in host_in.items():
+                t[k].copy_(v, non_blocking=True)
+            for dst, src in zip(idx_dev, idx_host):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for k, v in host_out.items():
+                v.copy_(dev_out[k], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        x0, x1 = ev(), ev()
+        x0.record(stream)
+        for _ in range(E):
+            e2e_step()
+        x1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = torch.tensor([x0.elapsed_time(x1) / E], device=dev)
+        if world > 1:
+            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * flops_step / (float(e2e_ms.item()) * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": float(e2e_ms.item()),
+               "note": "pinned host inputs copied in and all outputs/gradients copied out "
+                       "every step, same stream"}
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        th = {k: v.cpu() for k, v in t.items()}
+        p_cpu, s_cpu, n_s = time_oracle(st, th, 15.0, seed=7, n_rows=8)
+        cpu_base = {"value": p_cpu * 10 * d / s_cpu / 1e12, "unit": UNIT, "cores": blas_threads(),
+                    "kind": "oracle",
+                    "sample": f"{n_s} samples of 8 main + 24 branch rows of one random sequence, "
+                              f"all heads, fwd O/LSE + dQ in fp64 ({p_cpu} pairs, {s_cpu:.1f} s); "
+                              "dK/dV not computed, so this overstates CPU throughput"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(st, pairs, args.workload, in_bytes),
+            "pct_of_spec_bf16_peak": 100.0 * value / world / SPEC_BF16_TFLOPS,
+            "pct_of_measured_bf16_sustained": 100.0 * value / world / peak,
+            "fwd_kernel_ms": fwd_avg, "bwd_kernel_ms": bwd_avg, "plan_ms": plan_ms,
+            "fwd_tflops_4d": fwd_flops / (fwd_avg * 1e-3) / 1e12,
+            "fwd_bwd_tflops_14d": world * 14 * d * pairs / (ms_step * 1e-3) / 1e12,
+            "kernel_family": ba.ba_get_kernel_family(),
+            "roofline": {"bound": "tensor", "kernel": kernel_name, "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "traffic": traffic,
+                         "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside "
+                                        "the step loop)",
+                         "algorithmic": f"{'10' if dom == 'bwd' else '4'} d x {pairs} pairs "
+                                        "per launch"},
+            "cpu_baseline": cpu_base,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,239 @@
+/*
+ * branch_attn.h -- C ABI of the B200 (sm_100a) branch-attention library.
+ *
+ * What it computes ("Online Draft Co-Training", arXiv 2609.07108; paper
+ * summary pages, technical-contribution and method-detail sections): the
+ * attention layer of a speculative-decoding draft trained online next to its
+ * target.  Tokens are packed without padding.  Main tokens form sequences
+ * given by cu_seqlens; a main query attends causally to its own sequence.
+ * Each branch (an EAGLE-3 TTT chain, a DFlash block or a DSpark block) hangs
+ * off one main position, its anchor, and owns `depth` branch tokens with their
+ * own Q/K/V.  A branch query attends to
+ *   (1) the main keys of the anchor's sequence at positions <= anchor, and
+ *   (2) the keys of its own branch: depth <= own depth (TTT-causal,
+ *       block-causal) or the whole block (block-bidirectional),
+ * and the two partial results (O_m, l_m), (O_b, l_b) are merged by the
+ * online-softmax rule  l = log(e^{l_m} + e^{l_b}),
+ *                      O = e^{l_m - l} O_m + e^{l_b - l} O_b.
+ * The zigzag layout of the core-innovation section (each sequence cut into
+ * 2C chunks, shard i holding chunks i and 2C-1-i, branches staying with their
+ * anchor's shard) is available as a virtual shard order on one GPU: partial
+ * results of every ring step are merged by the same rule.
+ *
+ * Conventions for every call below
+ *   - Tensors are contiguous, row-major, bf16 unless stated:
+ *       Q, O, dO, dQ  [tokens, Hq,  d]
+ *       K, V, dK, dV  [tokens, Hkv, d]
+ *       LSE           [Hq, tokens] fp32, natural log, softmax scale included.
+ *     "_m" tensors cover the n_main main tokens, "_b" tensors the
+ *     n_branch_tokens branch tokens, stored anchor-major, depth-minor.
+ *   - q head h reads kv head h / (Hq / Hkv) (grouped-query attention).
+ *   - All pointers except the ba_problem struct itself are DEVICE pointers
+ *     owned by the caller; the library never allocates device memory and
+ *     keeps no pointer after a call returns.  Tensor pointers must be 16-byte
+ *     aligned (else BA_ERR_MISALIGNED), index arrays 4-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Host-side argument checks run before any launch; a
+ *     call that returns an error has launched nothing.
+ *   - Content checks of the index arrays (sorted anchors, depth range, ...)
+ *     run on the device inside ba_plan; they set a status word inside the
+ *     plan workspace, every later kernel that reads that plan returns without
+ *     touching its outputs when the word is non-zero, and ba_plan_status()
+ *     reads it back (synchronising the stream).
+ *   - Errors return a negative ba_status; ba_last_error() gives a message for
+ *     the calling thread's last failing call.
+ */
+#ifndef BRANCH_ATTN_H
+#define BRANCH_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BA_API __attribute__((visibility("default")))
+#else
+#define BA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *ba_stream_t;
+
+/* Branch-local mask kinds (research-background section: EAGLE-3 test-time
+ * training chains, DFlash block diffusion, DSpark Markov heads). */
+typedef enum {
+  BA_MASK_TTT_CAUSAL = 0,   /* depth j sees own-branch depths 0..j        */
+  BA_MASK_BLOCK_BIDIR = 1,  /* every block token sees the whole block     */
+  BA_MASK_BLOCK_CAUSAL = 2  /* block token j sees block tokens 0..j       */
+} ba_mask_kind;
+
+typedef enum {
+  BA_OK = 0,
+  BA_ERR_INVALID_ARG = -1,         /* bad size, enum, NULL pointer          */
+  BA_ERR_UNSUPPORTED = -2,         /* valid but not built (head_dim, GPU)  */
+  BA_ERR_MISALIGNED = -3,          /* pointer alignment violated           */
+  BA_ERR_WORKSPACE_TOO_SMALL = -4, /* caller's workspace below the query   */
+  BA_ERR_CUDA = -5,                /* a CUDA runtime call failed           */
+  BA_ERR_DEVICE_TIMEOUT = -6,      /* a bounded device-side wait gave up   */
+  BA_ERR_BAD_METADATA = -7         /* the plan's device-side checks failed */
+} ba_status;
+
+/* Device-side content-check bits reported by ba_plan_status(). */
+#define BA_META_CU_START 0x01       /* cu_seqlens[0] != 0                  */
+#define BA_META_CU_ORDER 0x02       /* cu_seqlens not strictly increasing  */
+#define BA_META_CU_TOTAL 0x04       /* cu_seqlens[n_seqs] != n_main        */
+#define BA_META_ANCHOR_RANGE 0x08   /* anchor outside [0, n_main)          */
+#define BA_META_ANCHOR_ORDER 0x10   /* anchors decrease                    */
+#define BA_META_DEPTH_RANGE 0x20    /* depth outside [1, 64]               */
+#define BA_META_DEPTH_TOTAL 0x40    /* sum(depth) != n_branch_tokens       */
+
+/* One packed batch.  The index arrays are device pointers, int32:
+ *   cu_seqlens    [n_seqs + 1], cu_seqlens[0] = 0, strictly increasing,
+ *                 cu_seqlens[n_seqs] = n_main
+ *   branch_anchor [n_branches], packed main index, non-decreasing
+ *   branch_depth  [n_branches], 1..64; sum = n_branch_tokens
+ * scale: softmax scale (> 0), usually 1/sqrt(head_dim).
+ * zigzag_C: 1 = monolithic; C > 1 = forward computed as C virtual zigzag
+ *   shards (2C chunks per sequence) whose ring-step partials are merged by
+ *   the LSE rule; the result equals the monolithic one up to rounding. */
+typedef struct {
+  int32_t n_seqs;
+  int32_t n_main;
+  int32_t n_branches;
+  int32_t n_branch_tokens;
+  int32_t hq;
+  int32_t hkv;
+  int32_t head_dim;      /* 64 or 128 */
+  float scale;
+  int32_t mask;          /* ba_mask_kind */
+  int32_t zigzag_C;      /* 1..64 */
+  const int32_t *cu_seqlens;
+  const int32_t *branch_anchor;
+  const int32_t *branch_depth;
+} ba_problem;
+
+/* Byte offsets of the metadata arrays inside a plan workspace (all int32).
+ * Query tiles are BA_TILE_M rows (main tiles first, then branch tiles), key
+ * tiles BA_TILE_N rows.
+ *   status      [4]           word 0 = OR of BA_META_* bits
+ *   cu_branch   [n_branches+1]  exclusive scan of branch_depth
+ *   branch_seq  [n_branches]    sequence holding each anchor
+ *   row_iv      [(n_main + n_branch_tokens) * 4]  per query row: first and
+ *               last visible main key, first and last visible branch-local
+ *               key row (empty = 0, -1); main rows first
+ *   qtile       [n_qtiles * 6]  kv_begin, full_begin, full_end, kv_end
+ *               (main key tiles; [full_begin, full_end) need no mask),
+ *               bl_begin, bl_end (branch-local key rows)
+ *   kv_main     [n_kv_main * 4]  main / branch query-tile ranges that visit
+ *               each main key tile (backward work list)
+ *   kv_branch   [n_kv_branch * 2]  branch query-tile range per branch key tile
+ *   fwd_order   [n_qtiles]       query tiles by decreasing cost
+ *   bwd_order   [n_kv_main + n_kv_branch]  key tiles by decreasing cost
+ *   fwd_cost, bwd_cost           the costs used for the two orders
+ *   zz_tiles    [zigzag_C * n_qtiles * 4]  (zigzag_C > 1 only) per ring step
+ *               and query tile, two key-tile ranges [b0, e0), [b1, e1)  */
+#define BA_TILE_M 128
+#define BA_TILE_N 128
+typedef struct {
+  size_t total_bytes;
+  size_t off_status, off_cu_branch, off_branch_seq, off_row_iv, off_qtile;
+  size_t off_kv_main, off_kv_branch, off_fwd_order, off_bwd_order;
+  size_t off_fwd_cost, off_bwd_cost, off_zz_tiles;
+  int32_t n_qtiles_main, n_qtiles_branch, n_kv_main, n_kv_branch;
+} ba_plan_layout;
+
+/* Workspace sizes for one problem (host-only; no device access).
+ * plan_bytes: the plan (metadata) workspace, written by ba_plan and read by
+ *   branch_attn_fwd / branch_attn_bwd.
+ * fwd_bytes:  scratch of branch_attn_fwd (0 when zigzag_C == 1; otherwise
+ *   fp32 accumulators of O and LSE for every query row and head).
+ * bwd_bytes:  scratch of branch_attn_bwd: D = rowsum(dO * O) fp32
+ *   [Hq, rows] and the fp32 dQ accumulator [rows, Hq, d]. */
+BA_API ba_status ba_workspace_size(const ba_problem *p, size_t *plan_bytes,
+                            size_t *fwd_bytes, size_t *bwd_bytes);
+
+/* Layout of the plan workspace (host-only). */
+BA_API ba_status ba_plan_layout_query(const ba_problem *p, ba_plan_layout *out);
+
+/* Builds the tile metadata on the device (method-detail section: which main
+ * keys and which branch keys each query sees).  Async on `stream`. */
+BA_API ba_status ba_plan(const ba_problem *p, void *plan_ws, size_t plan_bytes,
+                  ba_stream_t stream);
+
+/* Synchronises `stream` and returns the plan's content-check word
+ * (0 = valid) in *status_out; BA_ERR_BAD_METADATA when it is non-zero. */
+BA_API ba_status ba_plan_status(const void *plan_ws, ba_stream_t stream,
+                         int32_t *status_out);
+
+/* Forward.  Main rows: causal attention over their own sequence.  Branch
+ * rows: main prefix up to the anchor plus own branch, merged by the LSE rule
+ * (the branch-local partial is merged into the main partial in the kernel's
+ * epilogue).  Writes o_m, o_b (bf16) and lse_m [Hq, n_main],
+ * lse_b [Hq, n_branch_tokens] (fp32).  fwd_ws may be NULL when fwd_bytes is
+ * 0.  Requires a plan built by ba_plan for the same problem. */
+BA_API ba_status branch_attn_fwd(const ba_problem *p, const void *plan_ws,
+                          void *fwd_ws, size_t fwd_bytes,
+                          const void *q_m, const void *k_m, const void *v_m,
+                          const void *q_b, const void *k_b, const void *v_b,
+                          void *o_m, void *o_b, float *lse_m, float *lse_b,
+                          ba_stream_t stream);
+
+/* Backward of sum(O * dO): dQ, dK, dV for main and branch tokens.  P is
+ * recomputed from the merged LSE written by branch_attn_fwd (lse_m, lse_b),
+ * D = rowsum(dO * O) from the forward outputs.  dK/dV are summed over the q
+ * heads of each kv group.  All six gradient tensors are fully overwritten. */
+BA_API ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws,
+                          void *bwd_ws, size_t bwd_bytes,
+                          const void *q_m, const void *k_m, const void *v_m,
+                          const void *q_b, const void *k_b, const void *v_b,
+                          const void *o_m, const void *o_b,
+                          const float *lse_m, const float *lse_b,
+                          const void *do_m, const void *do_b,
+                          void *dq_m, void *dk_m, void *dv_m,
+                          void *dq_b, void *dk_b, void *dv_b,
+                          ba_stream_t stream);
+
+/* Standalone online-softmax merge (technical-contribution section):
+ *   l = log(e^{l_a} + e^{l_b}),  O = e^{l_a - l} O_a + e^{l_b - l} O_b.
+ * O_* are [rows, heads, head_dim] (fp32 when o_is_fp32, else bf16), l_*
+ * [heads, rows] fp32.  An empty partial (l = -inf) contributes nothing; two
+ * empty partials give O = 0, l = -inf.  o_out may alias o_a and lse_out may
+ * alias lse_a (in-place accumulation); other overlaps are undefined. */
+BA_API ba_status lse_merge(int64_t rows, int32_t heads, int32_t head_dim,
+                    int32_t o_is_fp32, const void *o_a, const float *lse_a,
+                    const void *o_b, const float *lse_b, void *o_out,
+                    float *lse_out, ba_stream_t stream);
+
+/* Kernel family for the attention kernels:
+ *   0 = default (tcgen05/TMEM/TMA kernels),
+ *   1 = tcgen05/TMEM/TMA kernels,
+ *   2 = warp-level mma.sync kernels (the pre-Blackwell tensor-core path, kept
+ *       as a second independent implementation).
+ * Returns BA_ERR_INVALID_ARG for other values.  Process-wide. */
+BA_API ba_status ba_set_kernel_family(int32_t family);
+BA_API int32_t ba_get_kernel_family(void);
+
+/* Benchmark instrumentation.  After ba_set_kernel_events(which, start, stop)
+ * every later call records the caller-owned CUDA event `start` (a cudaEvent_t)
+ * on the call's stream right before its attention kernel and `stop` right
+ * after it (which = 0: branch_attn_fwd, 1: branch_attn_bwd; for the zigzag
+ * forward the pair brackets all ring-step launches).  NULL events switch it
+ * off.  Process-wide; not for concurrent use from several threads. */
+BA_API ba_status ba_set_kernel_events(int32_t which, void *start_event, void *stop_event);
+
+/* Number of kernel launches the library has issued in this process. */
+BA_API int64_t ba_launch_count(void);
+
+/* Message for the calling thread's last failing call ("" if none). */
+BA_API const char *ba_last_error(void);
+
+/* Library version string. */
+BA_API const char *ba_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BRANCH_ATTN_H */

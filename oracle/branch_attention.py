@@ -309,11 +309,15 @@ def _row_sets(st, dv, main_rows, branch_rows):
 
 
 def rows_forward(st, t, main_rows=(), branch_rows=(), with_dq=False, heads=None):
-    """Forward (and optionally dQ) of selected query rows, each from its own key set.
+    """Forward (and optionally dQ) of selected query rows, each over its own key set.
 
     Returns dict with o [R, Hq, d], lse [Hq, R] and, if with_dq, dq [R, Hq, d],
     in the order main_rows then branch_rows.  Only q heads in `heads` (default:
     all) are computed; the others stay zero.
+
+    Rows reading the same sequence share one score matrix S = K_prefix q^T
+    (a plain matmul); each row then masks the keys it does not see (main keys
+    past its own position / anchor) and appends its branch-local scores.
     """
     dv = derive(st)
     items = _row_sets(st, dv, main_rows, branch_rows)
@@ -324,8 +328,6 @@ def rows_forward(st, t, main_rows=(), branch_rows=(), with_dq=False, heads=None)
     o = np.zeros((R, hq, d))
     lse = np.zeros((hq, R))
     dq = np.zeros((R, hq, d)) if with_dq else None
-    # A row's main keys are always a prefix [cu[s], hi] of one sequence, so
-    # rows are grouped by sequence and read views of one converted prefix.
     by_seq: Dict[int, List[int]] = {}
     for i, (kind, r, mk, lk) in enumerate(items):
         by_seq.setdefault(int(dv.main_seq[mk[0]]), []).append(i)
@@ -333,33 +335,43 @@ def rows_forward(st, t, main_rows=(), branch_rows=(), with_dq=False, heads=None)
     for s, idx in by_seq.items():
         lo = int(dv.cu[s])
         hi = max(int(items[i][2][-1]) for i in idx) + 1
+        nm = np.array([items[i][2].size for i in idx])            # main keys per row
+        assert all(items[i][2][0] == lo for i in idx)
+        visible = np.arange(hi - lo)[:, None] < nm[None, :]        # [L, R]
+        qs = np.stack([to64(t["q_" + ("m" if items[i][0] == "main" else "b")][items[i][1]])
+                       for i in idx])                              # [R, Hq, d]
+        dos = np.stack([to64(t["do_" + ("m" if items[i][0] == "main" else "b")][items[i][1]])
+                        for i in idx]) if with_dq else None
         for g in groups:
-            km = to64(t["k_m"][lo:hi, g])
+            km = to64(t["k_m"][lo:hi, g])                          # [L, d]
             vm = to64(t["v_m"][lo:hi, g])
-            for i in idx:
-                kind, r, mk, lk = items[i]
-                assert mk[0] == lo and mk[-1] == lo + mk.size - 1
-                nm = mk.size
-                sfx = "m" if kind == "main" else "b"
-                qx = to64(t["q_" + sfx][r])
-                dox = to64(t["do_" + sfx][r]) if with_dq else None
-                kl = to64(t["k_b"][lk, g]) if lk.size else np.zeros((0, d))
-                vl = to64(t["v_b"][lk, g]) if lk.size else np.zeros((0, d))
-                for h in heads:
-                    if h // grp != g:
-                        continue
-                    sc = st.scale * np.concatenate([km[:nm] @ qx[h], kl @ qx[h]])
-                    m = sc.max()
-                    p = np.exp(sc - m)
-                    z = p.sum()
-                    lse[h, i] = m + np.log(z)
-                    p = p / z
-                    o[i, h] = p[:nm] @ vm[:nm] + p[nm:] @ vl
-                    if with_dq:
-                        dp = np.concatenate([vm[:nm] @ dox[h], vl @ dox[h]])
-                        dd = float(dox[h] @ o[i, h])
-                        ds = p * (dp - dd)
-                        dq[i, h] = st.scale * (ds[:nm] @ km[:nm] + ds[nm:] @ kl)
+            kl = [to64(t["k_b"][items[i][3], g]) for i in idx]     # per-row local keys
+            vl = [to64(t["v_b"][items[i][3], g]) for i in idx]
+            for h in heads:
+                if h // grp != g:
+                    continue
+                sm = st.scale * (km @ qs[:, h, :].T)               # [L, R]
+                sm = np.where(visible, sm, -np.inf)
+                sl = [st.scale * (kl[c] @ qs[c, h]) for c in range(len(idx))]
+                m = np.maximum(sm.max(axis=0),
+                               np.array([x.max() if x.size else -np.inf for x in sl]))
+                pm = np.exp(sm - m[None, :])
+                pl = [np.exp(x - m[c]) for c, x in enumerate(sl)]
+                z = pm.sum(axis=0) + np.array([x.sum() for x in pl])
+                pm = pm / z[None, :]
+                pl = [x / z[c] for c, x in enumerate(pl)]
+                oo = pm.T @ vm + np.stack([pl[c] @ vl[c] for c in range(len(idx))])
+                for c, i in enumerate(idx):
+                    lse[h, i] = m[c] + np.log(z[c])
+                    o[i, h] = oo[c]
+                if with_dq:
+                    dpm = vm @ dos[:, h, :].T                      # [L, R]
+                    dd = (dos[:, h, :] * oo).sum(axis=1)
+                    dsm = pm * (dpm - dd[None, :])
+                    dqm = st.scale * (dsm.T @ km)
+                    for c, i in enumerate(idx):
+                        dsl = pl[c] * (vl[c] @ dos[c, h] - dd[c])
+                        dq[i, h] = dqm[c] + st.scale * (dsl @ kl[c])
     out = {"o": o, "lse": lse}
     if with_dq:
         out["dq"] = dq
@@ -370,24 +382,29 @@ def rows_backward_dq(st, t, main_rows=(), branch_rows=(), heads=None):
     return rows_forward(st, t, main_rows, branch_rows, with_dq=True, heads=heads)
 
 
-def keys_backward(st, t, main_keys=(), branch_keys=()):
-    """dK and dV of selected key rows: every query that sees them, in full.
+def keys_backward(st, t, main_keys=(), branch_keys=(), groups=None):
+    """dK and dV of selected key rows, summed over every query that sees them.
 
+    P_ik = exp(S_ik - l_i) needs only q_i, k and the query's LSE l_i, which
+    rows_forward gives (with O_i for D_i = dO_i . O_i); so each query scores
+    just the selected keys it sees: dV_k += P_ik dO_i, dK_k += scale dS_ik q_i,
+    dS_ik = P_ik (dO_i . v_k - D_i).
     Returns dict with dk_m/dv_m [len(main_keys), Hkv, d] and dk_b/dv_b
-    [len(branch_keys), Hkv, d].
+    [len(branch_keys), Hkv, d]; only kv heads in `groups` (default: all) are
+    computed, each summed over all q heads of its group.
     """
     dv = derive(st)
-    n, nb = dv.n_main, dv.n_branch_tokens
     hq, hkv, d = st.hq, st.hkv, st.head_dim
     grp = hq // hkv
-    main_keys = [int(k) for k in main_keys]
-    branch_keys = [int(k) for k in branch_keys]
+    groups = list(range(hkv)) if groups is None else [int(g) for g in groups]
+    heads = [h for h in range(hq) if h // grp in groups]
+    main_keys = np.asarray([int(k) for k in main_keys], dtype=np.int64)
+    branch_keys = np.asarray([int(k) for k in branch_keys], dtype=np.int64)
     anchors = np.asarray(st.anchors, dtype=np.int64)
-    # queries that see any selected key
     q_main, q_branch = set(), set()
     for k in main_keys:
         s = dv.main_seq[k]
-        q_main.update(range(k, int(dv.cu[s + 1])))
+        q_main.update(range(int(k), int(dv.cu[s + 1])))
         for b in np.nonzero((anchors >= k) & (dv.branch_seq == s))[0]:
             q_branch.update(range(int(dv.cu_branch[b]), int(dv.cu_branch[b + 1])))
     for k in branch_keys:
@@ -395,54 +412,54 @@ def keys_backward(st, t, main_keys=(), branch_keys=()):
         q_branch.update(range(int(dv.cu_branch[b]), int(dv.cu_branch[b + 1])))
     q_main = sorted(q_main)
     q_branch = sorted(q_branch)
-    fw = rows_forward(st, t, q_main, q_branch)
+    fw = rows_forward(st, t, q_main, q_branch, heads=heads)
     items = _row_sets(st, dv, q_main, q_branch)
-    mk_pos = {k: i for i, k in enumerate(main_keys)}
-    bk_pos = {k: i for i, k in enumerate(branch_keys)}
-    dk_m = np.zeros((len(main_keys), hkv, d))
-    dv_m = np.zeros((len(main_keys), hkv, d))
-    dk_b = np.zeros((len(branch_keys), hkv, d))
-    dv_b = np.zeros((len(branch_keys), hkv, d))
+    km_sel = to64(t["k_m"][main_keys]) if main_keys.size else np.zeros((0, hkv, d))
+    vm_sel = to64(t["v_m"][main_keys]) if main_keys.size else np.zeros((0, hkv, d))
+    kb_sel = to64(t["k_b"][branch_keys]) if branch_keys.size else np.zeros((0, hkv, d))
+    vb_sel = to64(t["v_b"][branch_keys]) if branch_keys.size else np.zeros((0, hkv, d))
+    dk_m = np.zeros((main_keys.size, hkv, d))
+    dv_m = np.zeros((main_keys.size, hkv, d))
+    dk_b = np.zeros((branch_keys.size, hkv, d))
+    dv_b = np.zeros((branch_keys.size, hkv, d))
     for i, (kind, r, mk, lk) in enumerate(items):
-        sel_m = [(j, mk_pos[int(k)]) for j, k in enumerate(mk) if int(k) in mk_pos]
-        sel_b = [(j, bk_pos[int(k)]) for j, k in enumerate(lk) if int(k) in bk_pos]
-        if not sel_m and not sel_b:
+        sel_m = np.nonzero((main_keys >= mk[0]) & (main_keys <= mk[-1]))[0]
+        sel_b = (np.nonzero((branch_keys >= lk[0]) & (branch_keys <= lk[-1]))[0]
+                 if lk.size else np.zeros(0, dtype=np.int64))
+        if sel_m.size == 0 and sel_b.size == 0:
             continue
-        qx = to64(t["q_" + ("m" if kind == "main" else "b")][r])
-        dox = to64(t["do_" + ("m" if kind == "main" else "b")][r])
-        kk = np.concatenate([to64(t["k_m"][mk]), to64(t["k_b"][lk]) if lk.size
-                             else np.zeros((0, hkv, d))], axis=0)
-        vv = np.concatenate([to64(t["v_m"][mk]), to64(t["v_b"][lk]) if lk.size
-                             else np.zeros((0, hkv, d))], axis=0)
-        for h in range(hq):
+        sfx = "m" if kind == "main" else "b"
+        qx = to64(t["q_" + sfx][r])
+        dox = to64(t["do_" + sfx][r])
+        for h in heads:
             g = h // grp
-            sc = st.scale * (kk[:, g, :] @ qx[h])
-            p = np.exp(sc - fw["lse"][h, i])
-            dp = vv[:, g, :] @ dox[h]
             dd = float(dox[h] @ fw["o"][i, h])
-            ds = p * (dp - dd)
-            for j, pos in sel_m:
-                dv_m[pos, g] += p[j] * dox[h]
-                dk_m[pos, g] += st.scale * ds[j] * qx[h]
-            off = mk.size
-            for j, pos in sel_b:
-                dv_b[pos, g] += p[off + j] * dox[h]
-                dk_b[pos, g] += st.scale * ds[off + j] * qx[h]
+            for sel, ksel, vsel, dk, dvv in ((sel_m, km_sel, vm_sel, dk_m, dv_m),
+                                            (sel_b, kb_sel, vb_sel, dk_b, dv_b)):
+                if sel.size == 0:
+                    continue
+                p = np.exp(st.scale * (ksel[sel, g] @ qx[h]) - fw["lse"][h, i])
+                ds = p * (vsel[sel, g] @ dox[h] - dd)
+                dvv[sel, g] += p[:, None] * dox[h][None]
+                dk[sel, g] += st.scale * ds[:, None] * qx[h][None]
     return {"dk_m": dk_m, "dv_m": dv_m, "dk_b": dk_b, "dv_b": dv_b}
 
 
 def useful_pairs(st) -> int:
-    """Number of unmasked (query head, key) pairs, summed over all q heads."""
+    """Number of unmasked (query head, key) pairs, summed over all q heads.
+
+    Main row r of sequence s: r - cu[s] + 1 keys.  Branch token j of branch b
+    (anchor a in sequence s, depth D): a - cu[s] + 1 main keys plus j + 1
+    (causal kinds) or D (block-bidirectional) branch keys.
+    """
     dv = derive(st)
-    total = 0
-    for r in range(dv.n_main):
-        total += r - int(dv.cu[dv.main_seq[r]]) + 1
+    main = int((np.arange(dv.n_main) - dv.cu[dv.main_seq] + 1).sum())
     anchors = np.asarray(st.anchors, dtype=np.int64)
-    for b in range(anchors.shape[0]):
-        a = int(anchors[b])
-        main = a - int(dv.cu[dv.branch_seq[b]]) + 1
-        depth = int(dv.cu_branch[b + 1] - dv.cu_branch[b])
-        for j in range(depth):
-            loc = depth if st.mask_kind == MASK_BLOCK_BIDIR else j + 1
-            total += main + loc
-    return total * st.hq
+    depth = dv.cu_branch[1:] - dv.cu_branch[:-1]
+    pre = anchors - dv.cu[dv.branch_seq] + 1 if anchors.size else np.zeros(0, dtype=np.int64)
+    if st.mask_kind == MASK_BLOCK_BIDIR:
+        loc = depth * depth
+    else:
+        loc = depth * (depth + 1) // 2
+    branch = int((pre * depth + loc).sum())
+    return (main + branch) * st.hq

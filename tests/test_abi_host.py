@@ -1,0 +1,156 @@
+"""Host-only checks of the C ABI: exports match the header, and every invalid
+argument is rejected with its documented status before anything launches.
+
+No call here reaches a kernel: every argument set is one the host-side
+validation rejects (fake device addresses are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import speculative_draft_branch_b200 as ba
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "branch_attn.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^BA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("ba_plan", "branch_attn_fwd", "branch_attn_bwd", "lse_merge",
+                     "ba_workspace_size", "ba_plan_status", "ba_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(ba.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(ba.EXPORTS) <= set(_declared())
+
+
+def _problem(**kw):
+    base = dict(n_seqs=2, n_main=256, n_branches=256, n_branch_tokens=768, hq=4, hkv=2,
+                head_dim=64, scale=0.125, mask=0, zigzag_C=1, cu_seqlens=0x10000,
+                branch_anchor=0x20000, branch_depth=0x30000)
+    base.update(kw)
+    return ba.BAProblem(**base)
+
+
+def _sizes(p):
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    st = ba.lib.ba_workspace_size(ctypes.byref(p), ctypes.byref(a), ctypes.byref(b),
+                                  ctypes.byref(c))
+    return st, a.value, b.value, c.value
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_seqs=0), -1), (dict(n_main=0), -1), (dict(n_seqs=300), -1),
+    (dict(n_branches=-1), -1), (dict(n_branch_tokens=100), -1),  # < n_branches
+    (dict(n_branch_tokens=256 * 65), -1),                         # depth > 64
+    (dict(hq=6, hkv=4), -1), (dict(hkv=0), -1), (dict(head_dim=96), -2),
+    (dict(head_dim=256), -2), (dict(mask=3), -1), (dict(mask=-1), -1),
+    (dict(zigzag_C=0), -1), (dict(zigzag_C=65), -1), (dict(scale=0.0), -1),
+    (dict(scale=float("nan")), -1), (dict(scale=float("inf")), -1),
+])
+def test_invalid_problem_rejected(kw, code):
+    st, *_ = _sizes(_problem(**kw))
+    assert st == code
+    assert ba.lib.ba_last_error().decode() != ""
+
+
+def test_workspace_sizes_follow_the_layout():
+    p = _problem()
+    st, plan_b, fwd_b, bwd_b = _sizes(p)
+    assert st == 0
+    L = ba.BAPlanLayout()
+    assert ba.lib.ba_plan_layout_query(ctypes.byref(p), ctypes.byref(L)) == 0
+    assert L.total_bytes == plan_b
+    assert (L.n_qtiles_main, L.n_qtiles_branch, L.n_kv_main, L.n_kv_branch) == (2, 6, 2, 6)
+    assert fwd_b == 0
+    rows = 256 + 768
+    assert bwd_b >= 4 * rows * 4 + 4 * rows * 4 * 64
+    # arrays are 256-byte aligned and do not overlap
+    offs = sorted(getattr(L, f) for f, _ in ba.BAPlanLayout._fields_ if f.startswith("off_"))
+    assert all(o % 256 == 0 for o in offs)
+    assert L.off_row_iv - L.off_branch_seq >= 4 * 256
+    pz = _problem(zigzag_C=8)
+    _, _, fwd_z, _ = _sizes(pz)
+    assert fwd_z >= 4 * rows * 4 * 64 + 4 * rows * 4
+
+
+def test_plan_rejects_bad_pointers_and_small_workspace():
+    p = _problem()
+    st, plan_b, _, _ = _sizes(p)
+    # NULL index arrays
+    q = _problem(cu_seqlens=None)
+    assert ba.lib.ba_plan(ctypes.byref(q), 0x100000, plan_b, None) == -1
+    # misaligned index array
+    q = _problem(branch_anchor=0x20002)
+    assert ba.lib.ba_plan(ctypes.byref(q), 0x100000, plan_b, None) == -3
+    # NULL / misaligned workspace
+    assert ba.lib.ba_plan(ctypes.byref(p), None, plan_b, None) == -1
+    assert ba.lib.ba_plan(ctypes.byref(p), 0x100008, plan_b, None) == -3
+    # workspace too small
+    assert ba.lib.ba_plan(ctypes.byref(p), 0x100000, plan_b - 1, None) == -4
+    assert "too small" in ba.lib.ba_last_error().decode()
+
+
+def test_fwd_bwd_reject_misaligned_or_missing_tensors():
+    p = _problem()
+    good = [0x200000 + i * 0x100000 for i in range(10)]
+    args = [ctypes.byref(p), 0x100000, None, 0] + good[:6] + good[6:8] + [0x900000, 0xa00000]
+    bad = list(args)
+    bad[4] = 0x200001  # q_m misaligned
+    assert ba.lib.branch_attn_fwd(*bad, None) == -3
+    bad = list(args)
+    bad[7] = None      # q_b missing while branch tokens exist
+    assert ba.lib.branch_attn_fwd(*bad, None) == -1
+    bad = list(args)
+    bad[12] = 0x900002  # lse_m not 4-byte aligned
+    assert ba.lib.branch_attn_fwd(*bad, None) == -3
+    # zigzag needs a workspace
+    pz = _problem(zigzag_C=4)
+    zargs = [ctypes.byref(pz), 0x100000, None, 0] + args[4:]
+    assert ba.lib.branch_attn_fwd(*zargs, None) == -1
+    zargs[2] = 0x5000000
+    zargs[3] = 16
+    assert ba.lib.branch_attn_fwd(*zargs, None) == -4
+    # backward: workspace too small, a gradient pointer missing
+    st, _, _, bwd_b = _sizes(p)
+    bargs = [ctypes.byref(p), 0x100000, 0x6000000, bwd_b - 256] + \
+        [0x200000 + i * 0x100000 for i in range(8)] + [0x900000, 0xa00000] + \
+        [0xb00000 + i * 0x100000 for i in range(8)]
+    assert ba.lib.branch_attn_bwd(*bargs, None) == -4
+    bargs[3] = bwd_b
+    bargs[16] = None  # dq_m
+    assert ba.lib.branch_attn_bwd(*bargs, None) == -1
+
+
+def test_lse_merge_rejections():
+    f = ba.lib.lse_merge
+    assert f(-1, 4, 64, 1, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == -1
+    assert f(10, 0, 64, 1, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == -1
+    assert f(10, 4, 80, 1, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == -2
+    assert f(10, 4, 64, 1, 0x1008, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == -3
+    assert f(10, 4, 64, 1, None, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == -1
+    assert f(10, 4, 64, 0, 0x1000, 0x2002, 0x3000, 0x4000, 0x5000, 0x6000, None) == -3
+    # zero rows is a no-op that touches nothing
+    assert f(0, 4, 64, 1, None, None, None, None, None, None, None) == 0
+
+
+def test_kernel_family_switch():
+    old = ba.ba_get_kernel_family()
+    try:
+        for fam in (0, 1, 2):
+            ba.ba_set_kernel_family(fam)
+            assert ba.ba_get_kernel_family() == fam
+        with pytest.raises(ba.BranchAttnError):
+            ba.ba_set_kernel_family(3)
+    finally:
+        ba.ba_set_kernel_family(old)

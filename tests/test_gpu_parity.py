@@ -1,0 +1,324 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (fp32 accumulation over bf16 inputs, P and dS rounded to bf16 for
+the tensor-core products): O, dQ, dK, dV max abs error <= 2e-2 and relative
+L2 error <= 1e-2 per tensor; LSE max abs error <= 1e-3; tile metadata
+bit-exact.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+ABS, REL, LSE_ABS = 2e-2, 1e-2, 1e-3
+KINDS = (wl.MASK_TTT_CAUSAL, wl.MASK_BLOCK_BIDIR, wl.MASK_BLOCK_CAUSAL)
+FAMILIES = (0, 2)   # 0 = default kernels (tcgen05 when built), 2 = mma.sync kernels
+
+
+def check(name, got, ref, abs_tol=ABS, rel_tol=REL):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    if got.size == 0:
+        return
+    assert np.isfinite(got).all(), f"{name}: non-finite values"
+    err = np.abs(got - ref).max()
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err <= abs_tol and rel <= rel_tol, f"{name}: max abs {err:.3e}, rel L2 {rel:.3e}"
+
+
+def check_lse(name, got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape
+    if got.size == 0:
+        return
+    err = np.abs(got - ref).max()
+    assert err <= LSE_ABS, f"{name}: LSE max abs {err:.3e}"
+
+
+def cpu(x):
+    return x.detach().float().cpu().numpy()
+
+
+def run(ba, st, t, family=0, bwd=True, zigzag_C=None):
+    ba.ba_set_kernel_family(family)
+    try:
+        prob = ba.Problem.from_structure(st, zigzag_C=zigzag_C)
+        runner = ba.BranchAttention(prob)
+        runner.plan()
+        assert runner.plan_status() == 0
+        out = runner.forward(t)
+        grads = runner.backward(t, out) if bwd else None
+        torch.cuda.synchronize()
+    finally:
+        ba.ba_set_kernel_family(0)
+    return runner, out, grads
+
+
+def full_parity(ba, st, seed, family):
+    t = wl.tensors(st, seed, "cuda")
+    _, out, g = run(ba, st, t, family)
+    o_m, o_b, lse_m, lse_b = oracle.forward_dense(st, t)
+    check("o_m", cpu(out["o_m"]), o_m)
+    check("o_b", cpu(out["o_b"]), o_b)
+    check_lse("lse_m", cpu(out["lse_m"]), lse_m)
+    check_lse("lse_b", cpu(out["lse_b"]), lse_b)
+    ref = oracle.backward_dense(st, t)
+    for name, r in zip(("dq_m", "dk_m", "dv_m", "dq_b", "dk_b", "dv_b"), ref):
+        check(name, cpu(g[name]), r)
+
+
+# ------------------------------------------------------------ metadata
+def _plan_equal(ba, st):
+    prob = ba.Problem.from_structure(st)
+    runner = ba.BranchAttention(prob)
+    runner.plan()
+    assert runner.plan_status() == 0
+    got = runner.read_plan()
+    ref = oracle.plan(st)
+    assert got["status"] == 0
+    for key, r in ref.items():
+        np.testing.assert_array_equal(got[key], r, err_msg=key)
+
+
+@pytest.mark.parametrize("name", wl.WORKLOADS)
+def test_plan_bit_exact_workloads(cuda_lib, name):
+    _plan_equal(cuda_lib, wl.structure(name))
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("kind", KINDS)
+def test_plan_bit_exact_random(cuda_lib, seed, kind):
+    st = wl.random_structure(seed, n_seqs=1 + seed, max_len=700, max_depth=64 if seed % 2 else 7,
+                             mask_kind=kind, branch_prob=0.3, zigzag_C=1 + seed % 4)
+    _plan_equal(cuda_lib, st)
+
+
+def test_plan_reports_bad_metadata(cuda_lib):
+    ba = cuda_lib
+    dev = "cuda"
+    cases = {
+        0x10: ([0, 10, 20], [5, 3], [2, 2]),     # anchors decrease
+        0x08: ([0, 10, 20], [5, 20], [2, 2]),    # anchor out of range
+        0x20: ([0, 10, 20], [5, 6], [0, 4]),     # depth 0
+        0x02: ([0, 10, 10], [5, 6], [2, 2]),     # empty sequence
+    }
+    for bit, (cu, an, de) in cases.items():
+        prob = ba.Problem(torch.tensor(cu, dtype=torch.int32, device=dev),
+                          torch.tensor(an, dtype=torch.int32, device=dev),
+                          torch.tensor(de, dtype=torch.int32, device=dev), 4, 2, 1, 64)
+        runner = ba.BranchAttention(prob)
+        runner.plan()
+        status = runner.plan_status()
+        assert status & bit, (bit, status)
+        # kernels reading a bad plan return without touching their outputs
+        st = wl.Structure("bad", np.array(cu), np.array(an), np.array([2, 2]), 2, 1, 64, 0)
+        t = wl.tensors(st, 0, dev)
+        out = runner.alloc_outputs()
+        for v in out.values():
+            v.fill_(7.0)
+        runner.forward(t, out)
+        torch.cuda.synchronize()
+        assert bool((out["o_m"] == 7.0).all()) and bool((out["lse_m"] == 7.0).all())
+
+
+# ------------------------------------------------------------ full parity
+@pytest.mark.parametrize("family", FAMILIES)
+def test_tiny_ttt_full(cuda_lib, family):
+    st = wl.structure("tiny_ttt")
+    full_parity(cuda_lib, st, wl.workload_seed("tiny_ttt"), family)
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("d,hq,hkv", [(64, 4, 2), (128, 4, 1), (128, 2, 2)])
+def test_random_full(cuda_lib, family, kind, d, hq, hkv):
+    """Several query and key tiles, ragged tails, varlen packing, GQA."""
+    st = wl.random_structure(10 + d + hq, n_seqs=3, max_len=330, max_depth=9, hq=hq, hkv=hkv,
+                             head_dim=d, mask_kind=kind, branch_prob=0.45)
+    full_parity(cuda_lib, st, 7, family)
+
+
+EDGE = {
+    "one_token": (np.array([0, 1]), np.array([0]), np.array([1])),
+    "no_branches": (np.array([0, 130, 131, 300]), np.zeros(0, int), np.zeros(0, int)),
+    "unit_sequences": (np.arange(0, 41), np.arange(0, 40, 3), np.full(14, 2)),
+    "depth64": (np.array([0, 70, 200]), np.array([0, 69, 70, 150, 199]), np.full(5, 64)),
+    "same_anchor": (np.array([0, 257]), np.full(9, 256), np.array([1, 2, 3, 4, 5, 6, 7, 8, 9])),
+    "first_positions": (np.array([0, 129, 258, 387]), np.array([0, 129, 258]),
+                        np.array([16, 16, 16])),
+}
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+@pytest.mark.parametrize("case", sorted(EDGE))
+@pytest.mark.parametrize("kind", KINDS)
+def test_edge_cases(cuda_lib, family, case, kind):
+    cu, an, de = EDGE[case]
+    st = wl.Structure(case, cu, an, de, 4, 2, 64, kind)
+    full_parity(cuda_lib, st, 3, family)
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+@pytest.mark.parametrize("C", [2, 3, 5])
+def test_zigzag_small_matches_oracle(cuda_lib, family, C):
+    """The virtual zigzag ring (C shards, LSE-merged) equals the monolithic result."""
+    st = wl.random_structure(21 + C, n_seqs=3, max_len=500, max_depth=5, hq=4, hkv=2,
+                             head_dim=64, branch_prob=0.5, zigzag_C=C)
+    t = wl.tensors(st, 5, "cuda")
+    _, out, _ = run(cuda_lib, st, t, family, bwd=False)
+    o_m, o_b, lse_m, lse_b = oracle.zigzag_forward(st, t, C)
+    check("o_m", cpu(out["o_m"]), o_m)
+    check("o_b", cpu(out["o_b"]), o_b)
+    check_lse("lse_m", cpu(out["lse_m"]), lse_m)
+    check_lse("lse_b", cpu(out["lse_b"]), lse_b)
+
+
+# ------------------------------------------------------------ lse_merge
+@pytest.mark.parametrize("fp32", [True, False])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("inplace", [False, True])
+def test_lse_merge(cuda_lib, fp32, d, inplace):
+    ba = cuda_lib
+    rows, heads = 1000, 3
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1)
+    dt = torch.float32 if fp32 else torch.bfloat16
+    oa = torch.randn(rows, heads, d, generator=gen, device="cuda").to(dt)
+    ob = torch.randn(rows, heads, d, generator=gen, device="cuda").to(dt)
+    la = torch.randn(heads, rows, generator=gen, device="cuda") * 5
+    lb = torch.randn(heads, rows, generator=gen, device="cuda") * 5
+    la[0, :50] = -float("inf")
+    lb[1, :50] = -float("inf")
+    la[2, :20] = -float("inf")
+    lb[2, :20] = -float("inf")
+    la[2, 20:40] = 80.0
+    lb[2, 20:40] = 80.5
+    ref_o, ref_l = oracle.lse_merge(cpu(oa).transpose(1, 0, 2), cpu(la),
+                                    cpu(ob).transpose(1, 0, 2), cpu(lb))
+    if inplace:
+        oo, lo = oa, la
+    else:
+        oo, lo = torch.empty_like(oa), torch.empty_like(la)
+    ba.lse_merge(oa, la, ob, lb, oo, lo)
+    torch.cuda.synchronize()
+    got_l = cpu(lo)
+    assert np.array_equal(np.isneginf(got_l), np.isneginf(ref_l))
+    fin = np.isfinite(ref_l)
+    assert np.abs(got_l[fin] - ref_l[fin]).max() <= 1e-5 * 100
+    tol = 1e-5 if fp32 else 1e-2
+    np.testing.assert_allclose(cpu(oo).transpose(1, 0, 2), ref_o, atol=tol, rtol=tol)
+
+
+# ------------------------------------------------------------ full-size workloads
+def _sample_rows(st, n_rand, rng):
+    dv = oracle.derive(st)
+    n, nb = dv.n_main, dv.n_branch_tokens
+    main = set()
+    for s in range(st.n_seqs):
+        main.update({int(dv.cu[s]), int(dv.cu[s + 1]) - 1})
+    main.update({127, 128, n - 1})
+    main.update(int(x) for x in rng.integers(0, n, n_rand))
+    branch = {0, nb - 1, min(127, nb - 1), min(128, nb - 1)}
+    branch.update(int(x) for x in rng.integers(0, nb, n_rand))
+    return sorted(x for x in main if 0 <= x < n), sorted(x for x in branch if 0 <= x < nb)
+
+
+def _count_visible(st):
+    iv = oracle.row_intervals(st)
+    cnt = (iv[:, 1] - iv[:, 0] + 1) + np.maximum(iv[:, 3] - iv[:, 2] + 1, 0)
+    return cnt[:st.n_main], cnt[st.n_main:]
+
+
+def workload_check(ba, st, seed, n_rand=24, tail_keys=128, groups=(0,), zigzag=False):
+    rng = np.random.default_rng(seed)
+    t = wl.tensors(st, seed, "cuda")
+    runner, out, g = run(ba, st, t, 0)
+    # 1) sampled rows: O, LSE and dQ over all heads
+    mr, br = _sample_rows(st, n_rand, rng)
+    ref = oracle.rows_backward_dq(st, t, mr, br)
+    R = len(mr)
+    check("o_m rows", cpu(out["o_m"][mr]), ref["o"][:R])
+    check("o_b rows", cpu(out["o_b"][br]), ref["o"][R:])
+    check_lse("lse_m rows", cpu(out["lse_m"][:, mr]), ref["lse"][:, :R])
+    check_lse("lse_b rows", cpu(out["lse_b"][:, br]), ref["lse"][:, R:])
+    check("dq_m rows", cpu(g["dq_m"][mr]), ref["dq"][:R])
+    check("dq_b rows", cpu(g["dq_b"][br]), ref["dq"][R:])
+    # 2) branch keys of a few branches (each seen by <= 64 queries)
+    dv = oracle.derive(st)
+    bsel = sorted({0, st.n_branches - 1, *rng.integers(0, st.n_branches, 3).tolist()})
+    bkeys = [k for b in bsel for k in range(int(dv.cu_branch[b]), int(dv.cu_branch[b + 1]))]
+    kb = oracle.keys_backward(st, t, branch_keys=bkeys, groups=groups)
+    gs = list(groups)
+    check("dk_b keys", cpu(g["dk_b"][bkeys][:, gs]), kb["dk_b"][:, gs])
+    check("dv_b keys", cpu(g["dv_b"][bkeys][:, gs]), kb["dv_b"][:, gs])
+    # 3) tail window of main keys of the shortest sequence
+    if tail_keys:
+        lens = np.diff(st.cu_seqlens)
+        s = int(np.argmin(lens))
+        hi = int(st.cu_seqlens[s + 1])
+        mkeys = list(range(max(int(st.cu_seqlens[s]), hi - tail_keys), hi))
+        km = oracle.keys_backward(st, t, main_keys=mkeys, groups=groups)
+        check("dk_m tail", cpu(g["dk_m"][mkeys][:, gs]), km["dk_m"][:, gs])
+        check("dv_m tail", cpu(g["dv_m"][mkeys][:, gs]), km["dv_m"][:, gs])
+    # 4) every row: with Q = 0 all visible scores are 0, so LSE = ln(#visible keys)
+    tz = dict(t)
+    tz["q_m"] = torch.zeros_like(t["q_m"])
+    tz["q_b"] = torch.zeros_like(t["q_b"])
+    zout = runner.forward(tz)
+    torch.cuda.synchronize()
+    cm, cb = _count_visible(st)
+    check_lse("lse_m (Q=0, all rows)", cpu(zout["lse_m"]), np.log(cm)[None].repeat(st.hq, 0))
+    check_lse("lse_b (Q=0, all rows)", cpu(zout["lse_b"]), np.log(cb)[None].repeat(st.hq, 0))
+    # 5) zigzag virtual shards agree with the monolithic run
+    if zigzag:
+        _, zo, _ = run(ba, st, t, 0, bwd=False, zigzag_C=st.zigzag_C)
+        for key in ("o_m", "o_b"):
+            check(f"{key} zigzag vs monolithic", cpu(zo[key]), cpu(out[key]))
+        for key in ("lse_m", "lse_b"):
+            check_lse(f"{key} zigzag vs monolithic", cpu(zo[key]), cpu(out[key]))
+        check("o_m rows (zigzag)", cpu(zo["o_m"][mr]), ref["o"][:R])
+        check("o_b rows (zigzag)", cpu(zo["o_b"][br]), ref["o"][R:])
+    return t
+
+
+@pytest.mark.parametrize("name", ["ttt_20k", "dflash_32k", "dspark_64k"])
+def test_workload_full_size(cuda_lib, name):
+    st = wl.structure(name)
+    workload_check(cuda_lib, st, wl.workload_seed(name))
+
+
+def test_workload_ttt_256k_and_zigzag(cuda_lib):
+    st = wl.structure("ttt_256k")
+    workload_check(cuda_lib, st, wl.workload_seed("ttt_256k"), n_rand=8, tail_keys=0,
+                   zigzag=True)
+
+
+def test_workload_ttt_256k_truncated_prefix(cuda_lib):
+    """First 8,192 tokens (and their branches) of the 256K batch, same data."""
+    full = wl.structure("ttt_256k")
+    st = dataclasses.replace(wl.truncate(full, 8192), zigzag_C=1)
+    t_full = wl.tensors(full, wl.workload_seed("ttt_256k"), "cuda")
+    t = {k: v.contiguous() for k, v in wl.slice_tensors(full, st, t_full).items()}
+    del t_full
+    torch.cuda.empty_cache()
+    _, out, g = run(cuda_lib, st, t, 0)
+    rng = np.random.default_rng(0)
+    mr, br = _sample_rows(st, 16, rng)
+    ref = oracle.rows_backward_dq(st, t, mr, br)
+    R = len(mr)
+    check("o_m", cpu(out["o_m"][mr]), ref["o"][:R])
+    check("o_b", cpu(out["o_b"][br]), ref["o"][R:])
+    check("dq_m", cpu(g["dq_m"][mr]), ref["dq"][:R])
+    check("dq_b", cpu(g["dq_b"][br]), ref["dq"][R:])
+    mkeys = list(range(8192 - 128, 8192))
+    km = oracle.keys_backward(st, t, main_keys=mkeys, groups=[0, 7])
+    check("dk_m tail", cpu(g["dk_m"][mkeys][:, [0, 7]]), km["dk_m"][:, [0, 7]])
+    check("dv_m tail", cpu(g["dv_m"][mkeys][:, [0, 7]]), km["dv_m"][:, [0, 7]])

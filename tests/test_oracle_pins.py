@@ -376,3 +376,34 @@ def test_plan_matches_bruteforce(kind, seed, tile):
         for i in range(len(order) - 1):
             a, b = order[i], order[i + 1]
             assert cost[a] > cost[b] or (cost[a] == cost[b] and a < b)
+
+
+def test_zz_tiles_cover_every_ring_step_pair():
+    """Each (row, key) pair the zigzag ring computes at step s lies inside the
+    listed key tiles of the row's tile at step s, and every pair is computed at
+    exactly one step."""
+    st = wl.random_structure(6, n_seqs=3, max_len=45, max_depth=3, zigzag_C=3,
+                             branch_prob=0.5)
+    C, BM = 3, 8
+    zz = oracle.plan(st, BM, BM)["zz_tiles"]
+    dv = oracle.derive(st)
+    n = dv.n_main
+    chunks = oracle.zigzag_chunks(dv.cu, C)
+    mask = oracle.dense_mask(st)
+    n_mt = -(-n // BM)
+    for r in range(n + dv.n_branch_tokens):
+        own = r if r < n else int(st.anchors[dv.row_branch[r - n]])
+        s = int(dv.main_seq[own])
+        kc = next(k for k, (lo, hi) in enumerate(chunks[s]) if lo <= own < hi)
+        shard = kc if kc < C else 2 * C - 1 - kc
+        t = r // BM if r < n else n_mt + (r - n) // BM
+        seen = np.zeros(n, dtype=int)
+        for step in range(C):
+            j = (shard - step) % C
+            for w, ch in enumerate((j, 2 * C - 1 - j)):
+                lo, hi = chunks[s][ch]
+                keys = [k for k in range(lo, hi) if mask[r, k]]
+                seen[keys] += 1
+                for k in keys:
+                    assert zz[step, t, 2 * w] <= k // BM < zz[step, t, 2 * w + 1]
+        np.testing.assert_array_equal(seen, mask[r, :n].astype(int))
