@@ -1,9 +1,12 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
 
 Tolerances (fp32 accumulation over bf16 inputs, P and dS rounded to bf16 for
-the tensor-core products): O, dQ, dK, dV max abs error <= 2e-2 and relative
-L2 error <= 1e-2 per tensor; LSE max abs error <= 1e-3; tile metadata
-bit-exact.
+the tensor-core products, bf16 outputs): O, dQ, dK, dV elementwise
+|x - ref| <= 2e-2 + 1e-2 |ref| (max abs error 2e-2, relative 1e-2) and
+relative L2 error <= 1e-2 per tensor; LSE max abs error <= 1e-3; tile
+metadata bit-exact.  The relative part of the elementwise bound is what makes
+the bound attainable for bf16 outputs: rounding a value of magnitude >= 4 to
+bf16 alone moves it by up to 2^-9 |x| >= 7.8e-3.
 """
 import dataclasses
 
@@ -28,9 +31,12 @@ def check(name, got, ref, abs_tol=ABS, rel_tol=REL):
     if got.size == 0:
         return
     assert np.isfinite(got).all(), f"{name}: non-finite values"
-    err = np.abs(got - ref).max()
+    diff = np.abs(got - ref)
+    excess = (diff - (abs_tol + rel_tol * np.abs(ref))).max()
     rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
-    assert err <= abs_tol and rel <= rel_tol, f"{name}: max abs {err:.3e}, rel L2 {rel:.3e}"
+    assert excess <= 0 and rel <= rel_tol, \
+        f"{name}: max abs {diff.max():.3e}, worst excess over 2e-2+1e-2|ref| {excess:.3e}, " \
+        f"rel L2 {rel:.3e}"
 
 
 def check_lse(name, got, ref):
