@@ -304,6 +304,11 @@ def run_ours(args):
     fs, fe, bs, be = [ev() for _ in range(K)], [ev() for _ in range(K)], \
         [ev() for _ in range(K)], [ev() for _ in range(K)]
     e0, e1 = ev(), ev()
+    # torch creates events lazily: record each once so the handle exists before
+    # the library records it around its kernels
+    for e in fs + fe + bs + be:
+        e.record(stream)
+    torch.cuda.synchronize()
     clocks = ClockSampler(local_rank)
     clocks.start()
     launches0 = ba.ba_launch_count()
