@@ -196,6 +196,28 @@ BA_API ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws,
                           void *dq_b, void *dk_b, void *dv_b,
                           ba_stream_t stream);
 
+/* branch_attn_bwd for callers that cannot allocate device memory (no
+ * counterpart in the paper; an interface addition of this library).
+ * Some host programs manage all device memory themselves (a process that
+ * reserves its whole HBM budget in its own pool at start-up, or a plugin whose
+ * host forbids allocation at run time) and cannot cudaMalloc the backward
+ * workspace.  This call takes the same arguments as branch_attn_bwd minus the
+ * workspace and keeps its scratch (D and the fp32 dQ accumulator) in a
+ * 32 MiB array compiled into the library, which every GPU that loads the
+ * library holds until exit.  It allocates nothing.
+ *   - Problems whose backward scratch (see ba_workspace_size) exceeds 32 MiB
+ *     are rejected with BA_ERR_WORKSPACE_TOO_SMALL before any launch.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls on a device share the array; each call re-initialises what it
+ *     needs, but calls whose kernels overlap on the GPU race on it. */
+BA_API ba_status branch_attn_bwd_static_scratch(
+    const ba_problem *p, const void *plan_ws, const void *q_m, const void *k_m,
+    const void *v_m, const void *q_b, const void *k_b, const void *v_b, const void *o_m,
+    const void *o_b, const float *lse_m, const float *lse_b, const void *do_m,
+    const void *do_b, void *dq_m, void *dk_m, void *dv_m, void *dq_b, void *dk_b, void *dv_b,
+    ba_stream_t stream);
+
 /* Standalone online-softmax merge (technical-contribution section):
  *   l = log(e^{l_a} + e^{l_b}),  O = e^{l_a - l} O_a + e^{l_b - l} O_b.
  * O_* are [rows, heads, head_dim] (fp32 when o_is_fp32, else bf16), l_*

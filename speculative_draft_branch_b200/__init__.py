@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "BA_OK", -1: "BA_ERR_INVALID_ARG", -2: "BA_ERR_UNSUPPORTED",
 EXPORTS = ("ba_workspace_size", "ba_plan_layout_query", "ba_plan", "ba_plan_status",
            "branch_attn_fwd", "branch_attn_bwd", "lse_merge", "ba_set_kernel_family",
            "ba_get_kernel_family", "ba_set_kernel_events", "ba_launch_count", "ba_last_error",
-           "ba_version")
+           "ba_version", "branch_attn_bwd_static_scratch")
 
 
 class BAProblem(ctypes.Structure):
@@ -73,6 +73,7 @@ def _load() -> ctypes.CDLL:
         "ba_plan_status": [VP, VP, ctypes.POINTER(I32)],
         "branch_attn_fwd": [P, VP, VP, S] + [VP] * 10 + [VP],
         "branch_attn_bwd": [P, VP, VP, S] + [VP] * 18 + [VP],
+        "branch_attn_bwd_static_scratch": [P, VP] + [VP] * 18 + [VP],
         "lse_merge": [I64, I32, I32, I32, VP, VP, VP, VP, VP, VP, VP],
         "ba_set_kernel_family": [I32],
         "ba_get_kernel_family": [],
@@ -234,6 +235,31 @@ def branch_attn_bwd(problem: Problem, plan_ws, bwd_ws, q_m, k_m, v_m, q_b, k_b, 
                                _ptr(o_m), _ptr(o_b), _ptr(lse_m), _ptr(lse_b), _ptr(do_m),
                                _ptr(do_b), _ptr(dq_m), _ptr(dk_m), _ptr(dv_m), _ptr(dq_b),
                                _ptr(dk_b), _ptr(dv_b), _stream(stream)))
+
+
+def branch_attn_bwd_static_scratch(problem: Problem, plan_ws, q_m, k_m, v_m, q_b, k_b, v_b, o_m,
+                                   o_b, lse_m, lse_b, do_m, do_b, dq_m, dk_m, dv_m, dq_b, dk_b,
+                                   dv_b, stream=None) -> None:
+    """branch_attn_bwd without a workspace argument, for callers that cannot
+    allocate device memory: the scratch lives in a fixed 32 MiB array inside
+    the library (larger problems are rejected).  Calls that overlap on the GPU
+    share that array and must not run concurrently."""
+    import torch
+    sh = problem.shapes()
+    pairs = (("q_m", q_m, "q_m"), ("k_m", k_m, "k_m"), ("v_m", v_m, "v_m"), ("q_b", q_b, "q_b"),
+             ("k_b", k_b, "k_b"), ("v_b", v_b, "v_b"), ("o_m", o_m, "q_m"), ("o_b", o_b, "q_b"),
+             ("do_m", do_m, "q_m"), ("do_b", do_b, "q_b"), ("dq_m", dq_m, "q_m"),
+             ("dk_m", dk_m, "k_m"), ("dv_m", dv_m, "v_m"), ("dq_b", dq_b, "q_b"),
+             ("dk_b", dk_b, "k_b"), ("dv_b", dv_b, "v_b"))
+    for name, t, like in pairs:
+        _expect(t, sh[like], torch.bfloat16, name)
+    _expect(lse_m, sh["lse_m"], torch.float32, "lse_m")
+    _expect(lse_b, sh["lse_b"], torch.float32, "lse_b")
+    _check(lib.branch_attn_bwd_static_scratch(
+        ctypes.byref(problem.c), _ptr(plan_ws), _ptr(q_m), _ptr(k_m), _ptr(v_m), _ptr(q_b),
+        _ptr(k_b), _ptr(v_b), _ptr(o_m), _ptr(o_b), _ptr(lse_m), _ptr(lse_b), _ptr(do_m),
+        _ptr(do_b), _ptr(dq_m), _ptr(dk_m), _ptr(dv_m), _ptr(dq_b), _ptr(dk_b), _ptr(dv_b),
+        _stream(stream)))
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, stream=None) -> None:
