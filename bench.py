@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="ttt_20k")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profile-sized case: only the first N main tokens and their branches")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -275,6 +277,8 @@ def run_ours(args):
             dist.barrier()
 
     st = wl.structure(args.workload)
+    if args.tokens:
+        st = wl.truncate(st, args.tokens)
     t = wl.tensors(st, wl.workload_seed(args.workload) + 1000 * rank, dev)
     prob = ba.Problem.from_structure(st, device=dev)
     runner = ba.BranchAttention(prob, device=dev)
