@@ -164,7 +164,11 @@ BA_API ba_status ba_plan(const ba_problem *p, void *plan_ws, size_t plan_bytes,
                   ba_stream_t stream);
 
 /* Synchronises `stream` and returns the plan's content-check word
- * (0 = valid) in *status_out; BA_ERR_BAD_METADATA when it is non-zero. */
+ * (0 = valid) in *status_out; BA_ERR_BAD_METADATA when it is non-zero.  The
+ * workspace also carries a second word that kernels reading this plan set
+ * when one of their bounded waits on the device gave up (the kernel then
+ * returns early and its outputs are not valid); that case returns
+ * BA_ERR_DEVICE_TIMEOUT.  ba_plan clears both words. */
 BA_API ba_status ba_plan_status(const void *plan_ws, ba_stream_t stream,
                          int32_t *status_out);
 

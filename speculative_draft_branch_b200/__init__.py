@@ -194,7 +194,7 @@ def ba_plan_status(plan_ws, stream=None) -> int:
     word = ctypes.c_int32()
     st = lib.ba_plan_status(_ptr(plan_ws), _stream(stream), ctypes.byref(word))
     if st not in (0, -7):
-        _check(st)
+        _check(st)  # BA_ERR_DEVICE_TIMEOUT or a CUDA error raises
     return word.value
 
 

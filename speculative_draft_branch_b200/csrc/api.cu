@@ -205,10 +205,8 @@ ba_status check_plan_ws(const void *plan_ws) {
   return BA_OK;
 }
 
-bool use_sm100() {
-  const int f = g_family.load();
-  return f != 2 && sm100_available();
-}
+bool use_sm100_fwd() { return g_family.load() != 2 && sm100_fwd_available(); }
+bool use_sm100_bwd() { return g_family.load() != 2 && sm100_bwd_available(); }
 
 #define BA_TRY(expr)                   \
   do {                                 \
@@ -255,15 +253,19 @@ ba_status ba_plan(const ba_problem *p, void *plan_ws, size_t plan_bytes, ba_stre
 
 ba_status ba_plan_status(const void *plan_ws, ba_stream_t stream, int32_t *status_out) {
   BA_TRY(check_plan_ws(plan_ws));
-  int32_t word = 0;
-  BA_TRY(cuda_check(cudaMemcpyAsync(&word, plan_ws, sizeof(word), cudaMemcpyDeviceToHost,
+  int32_t words[2] = {0, 0};
+  BA_TRY(cuda_check(cudaMemcpyAsync(words, plan_ws, sizeof(words), cudaMemcpyDeviceToHost,
                                     (cudaStream_t)stream),
                     "ba_plan_status copy"));
   BA_TRY(cuda_check(cudaStreamSynchronize((cudaStream_t)stream), "ba_plan_status sync"));
-  if (status_out) *status_out = word;
-  if (word != 0) {
-    set_error("plan content checks failed (status 0x%x)", word);
+  if (status_out) *status_out = words[0];
+  if (words[0] != 0) {
+    set_error("plan content checks failed (status 0x%x)", words[0]);
     return BA_ERR_BAD_METADATA;
+  }
+  if (words[1] != 0) {
+    set_error("a bounded device-side wait gave up (sites 0x%x)", words[1]);
+    return BA_ERR_DEVICE_TIMEOUT;
   }
   return BA_OK;
 }
@@ -302,7 +304,7 @@ ba_status branch_attn_fwd(const ba_problem *p, const void *plan_ws, void *fwd_ws
   a.o_m = (__nv_bfloat16 *)o_m; a.o_b = (__nv_bfloat16 *)o_b;
   a.lse_m = lse_m; a.lse_b = lse_b;
   cudaStream_t s = (cudaStream_t)stream;
-  const bool sm100 = use_sm100();
+  const bool sm100 = use_sm100_fwd();
   auto launch = [&](const AttnParams &x) {
     return sm100 ? launch_fwd_sm100(x, s) : launch_fwd_mma(x, s);
   };
@@ -368,7 +370,7 @@ ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws, void *bwd_ws
   cudaStream_t s = (cudaStream_t)stream;
   BA_TRY(launch_bwd_preprocess(a, s));
   record_event(1, true, s);
-  BA_TRY(use_sm100() ? launch_bwd_sm100(a, s) : launch_bwd_mma(a, s));
+  BA_TRY(use_sm100_bwd() ? launch_bwd_sm100(a, s) : launch_bwd_mma(a, s));
   record_event(1, false, s);
   return launch_dq_convert(a, (__nv_bfloat16 *)dq_m, (__nv_bfloat16 *)dq_b, s);
 }

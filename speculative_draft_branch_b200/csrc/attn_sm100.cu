@@ -1,13 +1,508 @@
-// tcgen05 / TMEM / TMA branch-attention kernels for sm_100a.
+// Branch attention on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// Forward kernel: one CTA per (query tile of 128 rows, q head), 8 warps.
+//   warp 0      TMA producer: Q once, then a 2-stage ring of 128-key K/V tiles
+//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into TMEM (two S
+//               buffers, so S_{j+1} runs while tile j is in softmax), then
+//               O += P_j V_j with O accumulating in TMEM
+//   warp 2      TMEM allocation (512 columns: S0, S1, O)
+//   warps 4-7   softmax, one thread per query row (= TMEM lane): reads its S
+//               row, masks it with the row's key interval, keeps the running
+//               max / sum, writes P (bf16) into shared memory in the 128-byte
+//               swizzled K-major layout the MMA reads, and rescales its O row
+//               in TMEM only when the running max grew by more than 2^8.
+// Key tiles come from the plan: the main key tiles of the query tile, then
+// (branch tiles) the branch-local key rows.  Folding each tile's partial into
+// the running (O, l) is the online-softmax merge; the branch-local tiles come
+// last, so their fold is the paper's merge of (O_b, l_b) into (O_m, l_m)
+// ("Online Draft Co-Training", technical-contribution section).  The epilogue
+// normalises O and writes the LSE, or, on the zigzag ring path, merges the
+// step's partial into an fp32 accumulator by the same rule.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "internal.cuh"
+#include "sm100.cuh"
 
 namespace ba {
+namespace {
 
-bool sm100_available() { return false; }
+using namespace sm100;
+using bf16 = __nv_bfloat16;
 
-ba_status launch_fwd_sm100(const AttnParams &, cudaStream_t) {
-  set_error("tcgen05 forward kernel not built");
-  return BA_ERR_UNSUPPORTED;
+constexpr float kNegInf = -INFINITY;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct TensorMaps {
+  CUtensorMap q_m, q_b, k_m, v_m, k_b, v_b;
+};
+
+// ---- host: tensor maps -------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [rows, heads, d] bf16 -> 3-D map (d, heads, rows), box (64, 1, 128), 128-byte swizzle.
+ba_status make_map(CUtensorMap *m, const void *ptr, int64_t rows, int heads, int d) {
+  auto fn = encode_fn();
+  if (!fn) {
+    set_error("cuTensorMapEncodeTiled unavailable");
+    return BA_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return BA_ERR_CUDA;
+  }
+  return BA_OK;
+}
+
+// ---- device ---------------------------------------------------------------------
+template <int D>
+struct FwdSmem {
+  bf16 q[128 * D];        // D/64 boxes of [128 rows][64], 16 KB each
+  bf16 k[2][128 * D];
+  bf16 v[2][128 * D];
+  bf16 p[2][128 * 128];   // P: two [128 rows][64 keys] halves
+  uint64_t bar_q;
+  uint64_t bar_kv_full[2], bar_kv_empty[2];
+  uint64_t bar_s_full[2], bar_s_empty[2];
+  uint64_t bar_p_full[2];
+  uint64_t bar_o_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Seg {
+  int key0, n, kind, full_b, full_e;
+};
+
+struct TileSegs {
+  Seg s[3];
+  int total;
+  __device__ __forceinline__ void locate(int it, int &key0, int &kind, bool &full) const {
+    int si = 0, sub = it;
+    if (sub >= s[0].n) {
+      sub -= s[0].n;
+      si = 1;
+      if (sub >= s[1].n) {
+        sub -= s[1].n;
+        si = 2;
+      }
+    }
+    const Seg g = si == 0 ? s[0] : (si == 1 ? s[1] : s[2]);
+    key0 = g.key0 + sub * 128;
+    kind = g.kind;
+    full = kind == 0 && key0 >= g.full_b && key0 + 128 <= g.full_e;
+  }
+};
+
+__device__ __forceinline__ TileSegs make_segs(const AttnParams &a, int t, bool is_main) {
+  TileSegs ts;
+  int n = 0;
+  const int32_t *qt = a.plan.qtile + (int64_t)t * 6;
+  const int zz = a.zz_step;
+  if (zz < 0) {
+    const int k0 = qt[0] * 128, k1 = min(qt[3] * 128, a.n_main);
+    ts.s[n++] = {k0, (k1 - k0 + 127) / 128, 0, qt[1] * 128, qt[2] * 128};
+  } else if (zz < a.zz_C) {
+    const int32_t *z = a.plan.zz_tiles + ((int64_t)zz * a.n_qt + t) * 4;
+    for (int w = 0; w < 2; ++w) {
+      const int k0 = z[2 * w] * 128, k1 = min(z[2 * w + 1] * 128, a.n_main);
+      if (k1 > k0) ts.s[n++] = {k0, (k1 - k0 + 127) / 128, w, 0, 0};
+    }
+  }
+  if (!is_main && (zz < 0 || zz == a.zz_C)) {
+    const int b0 = qt[4], b1 = qt[5];
+    if (b1 > b0) ts.s[n++] = {b0, (b1 - b0 + 127) / 128, 2, 0, 0};
+  }
+  for (int i = n; i < 3; ++i) ts.s[i] = {0, 0, 2, 0, 0};
+  ts.total = ts.s[0].n + ts.s[1].n + ts.s[2].n;
+  return ts;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    fwd_sm100_kernel(const AttnParams a, const __grid_constant__ TensorMaps tm) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  FwdSmem<D> &sm = *reinterpret_cast<FwdSmem<D> *>(smem_raw + (((raw + 1023) & ~1023u) - raw));
+  if (a.plan.status[0] != 0) return;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int item = blockIdx.x;
+  const int t = a.plan.fwd_order[item / a.hq];
+  const int h = item % a.hq;
+  const int g = h / (a.hq / a.hkv);
+  const bool is_main = t < a.n_qt_main;
+  const int tt = is_main ? t : t - a.n_qt_main;
+  const int rows_total = is_main ? a.n_main : a.n_bt;
+  const int row0 = tt * 128;
+  const int nrows = min(128, rows_total - row0);
+  const int row_off = is_main ? 0 : a.n_main;
+  const TileSegs segs = make_segs(a, t, is_main);
+  const int total = segs.total;
+  int *status_word = a.plan.status + 1;
+  volatile int *abort_flag = &sm.abort_flag;
+
+  const uint32_t b_q = smem_u32(&sm.bar_q), b_o = smem_u32(&sm.bar_o_done);
+  if (threadIdx.x == 0) {
+    mbar_init(b_q, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&sm.bar_kv_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_kv_empty[s]), 1);
+      mbar_init(smem_u32(&sm.bar_s_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_s_empty[s]), 128);
+      mbar_init(smem_u32(&sm.bar_p_full[s]), 128);
+    }
+    mbar_init(b_o, 1);
+    sm.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t t_o = tmem + 256;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    const CUtensorMap *qmap = is_main ? &tm.q_m : &tm.q_b;
+    if (total > 0) {
+      mbar_expect_tx(b_q, 128 * D * 2);
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x)
+        tma_load_3d(smem_u32(sm.q) + x * 16384, qmap, b_q, x * 64, h, row0);
+    }
+    int issued = 0;
+    for (int j = 0; j < total; ++j) {
+      const int st = j & 1;
+      if (j >= 2 && !mbar_wait(smem_u32(&sm.bar_kv_empty[st]), ((j - 2) >> 1) & 1, abort_flag,
+                               status_word, 1))
+        break;
+      int key0, kind;
+      bool full;
+      segs.locate(j, key0, kind, full);
+      const CUtensorMap *km = kind == 2 ? &tm.k_b : &tm.k_m;
+      const CUtensorMap *vm = kind == 2 ? &tm.v_b : &tm.v_m;
+      const uint32_t bar = smem_u32(&sm.bar_kv_full[st]);
+      mbar_expect_tx(bar, 2 * 128 * D * 2);
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x) {
+        tma_load_3d(smem_u32(sm.k[st]) + x * 16384, km, bar, x * 64, g, key0);
+        tma_load_3d(smem_u32(sm.v[st]) + x * 16384, vm, bar, x * 64, g, key0);
+      }
+      ++issued;
+    }
+    // on abort: let the loads already issued land before the CTA exits
+    for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
+      mbar_wait(smem_u32(&sm.bar_kv_full[j & 1]), (j >> 1) & 1, abort_flag, status_word, 2);
+    if (total > 0) mbar_wait(b_q, 0, abort_flag, status_word, 2);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+    bool ok = total == 0 || mbar_wait(b_q, 0, abort_flag, status_word, 3);
+    const uint32_t q_s = smem_u32(sm.q);
+    auto issue_pv = [&](int i) -> bool {
+      const int pb = i & 1;
+      if (!mbar_wait(smem_u32(&sm.bar_p_full[pb]), (i >> 1) & 1, abort_flag, status_word, 4))
+        return false;
+      tc_fence_after();
+      const uint32_t p_s = smem_u32(sm.p[pb]), v_s = smem_u32(sm.v[pb]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint64_t ad = sdesc(p_s + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc(v_s + k * 2048, 16384, 1024);
+        mma_bf16(t_o, ad, bd, idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
+      }
+      mma_commit(b_o);
+      mma_commit(smem_u32(&sm.bar_kv_empty[pb]));
+      return true;
+    };
+    for (int j = 0; ok && j < total; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(smem_u32(&sm.bar_kv_full[st]), (j >> 1) & 1, abort_flag, status_word, 5) ||
+          (j >= 2 && !mbar_wait(smem_u32(&sm.bar_s_empty[st]), ((j - 2) >> 1) & 1, abort_flag,
+                                status_word, 6))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t k_s = smem_u32(sm.k[st]);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+        mma_bf16(tmem + st * 128, sdesc(q_s + off, 16, 1024), sdesc(k_s + off, 16, 1024),
+                 idesc_qk, k > 0 ? 1u : 0u);
+      }
+      mma_commit(smem_u32(&sm.bar_s_full[st]));
+      if (j >= 1 && !issue_pv(j - 1)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok && total > 0) issue_pv(total - 1);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int row = threadIdx.x - 128;
+    const bool valid = row < nrows;
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    int lo[3] = {0, 0, 0}, hi[3] = {-1, -1, -1};
+    const int zz = a.zz_step;
+    if (valid) {
+      const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[row_off + row0 + row];
+      if (zz < 0 || zz == a.zz_C) {
+        lo[0] = iv.x; hi[0] = iv.y;
+        lo[2] = iv.z; hi[2] = iv.w;
+      }
+      if (zz >= 0 && zz < a.zz_C) {
+        int s_lo = 0, s_hi = a.n_seqs;
+        while (s_lo < s_hi) {
+          const int mid = (s_lo + s_hi + 1) >> 1;
+          if (a.cu_seqlens[mid] <= iv.x) s_lo = mid; else s_hi = mid - 1;
+        }
+        const int64_t L = a.cu_seqlens[s_lo + 1] - iv.x;
+        const int64_t pos = iv.y - iv.x;
+        const int C = a.zz_C;
+        const int c = (int)((2 * C * (pos + 1) - 1) / L);
+        const int shard = c < C ? c : 2 * C - 1 - c;
+        const int jw = ((shard - zz) % C + C) % C;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int ch = w == 0 ? jw : 2 * C - 1 - jw;
+          lo[w] = max(iv.x + (int)((ch * L) / (2 * C)), iv.x);
+          hi[w] = min(iv.x + (int)(((ch + 1) * L) / (2 * C)) - 1, iv.y);
+        }
+      }
+    }
+    float m_used = kNegInf, l = 0.f;
+    bool ok = true;
+    const uint32_t p_row = row * 128;
+    const uint32_t swz = (uint32_t)(row & 7);
+    for (int j = 0; j < total; ++j) {
+      const int sb = j & 1;
+      // warp-uniform decisions: tcgen05.ld / st below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_s_full[sb]), (j >> 1) & 1,
+                                             abort_flag, status_word, 7))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      int key0, kind;
+      bool full;
+      segs.locate(j, key0, kind, full);
+      const int clo = kind == 0 ? lo[0] : (kind == 1 ? lo[1] : lo[2]);
+      const int chi = kind == 0 ? hi[0] : (kind == 1 ? hi[1] : hi[2]);
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tmem + lane_addr + sb * 128 + c * 32, reinterpret_cast<uint32_t *>(s) + c * 32);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.bar_s_empty[sb]));
+      float mx = kNegInf;
+      if (full && valid) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          s[c] *= a.scale_log2;
+          mx = fmaxf(mx, s[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int key = key0 + c;
+          s[c] = (key >= clo && key <= chi) ? s[c] * a.scale_log2 : kNegInf;
+          mx = fmaxf(mx, s[c]);
+        }
+      }
+      const float m_new = fmaxf(m_used, mx);
+      const bool need = m_new > m_used + kRescaleThreshold;
+      const float alpha = need ? ex2(m_used - m_new) : 1.f;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O holds PV_{j-1}: wait for it, then scale the rows that need it in
+        // TMEM (the whole warp takes part; other lanes scale by 1)
+        if (!__all_sync(0xffffffffu, mbar_wait(b_o, (j - 1) & 1, abort_flag, status_word, 8))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + lane_addr + c * 32, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(t_o + lane_addr + c * 32, o);
+        }
+        tc_wait_st();
+      }
+      if (need) {
+        l *= alpha;
+        m_used = m_new;
+      }
+      const float msub = m_used == kNegInf ? 0.f : m_used;
+      const uint32_t p_s = smem_u32(sm.p[sb]);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          float pv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            pv[e] = ex2(s[half * 64 + ch * 8 + e] - msub);
+            l += pv[e];
+          }
+          st_shared_v4(p_s + half * 16384 + p_row + ((ch ^ swz) << 4), pack_bf16(pv[0], pv[1]),
+                       pack_bf16(pv[2], pv[3]), pack_bf16(pv[4], pv[5]),
+                       pack_bf16(pv[6], pv[7]));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.bar_p_full[sb]));
+    }
+    if (ok && total > 0 &&
+        !__all_sync(0xffffffffu, mbar_wait(b_o, (total - 1) & 1, abort_flag, status_word, 9)))
+      ok = false;
+    tc_fence_after();
+
+    // ------------------------------------------------------------ epilogue
+    const bool empty = !(l > 0.f) || m_used == kNegInf;
+    float lse = empty ? kNegInf : (m_used + __log2f(l)) * kLn2;
+    const float inv = empty ? 0.f : 1.f / l;
+    const bool final_out = zz < 0 || zz == a.zz_C;
+    float wa = 0.f, wb = 1.f;
+    float *acc = nullptr;
+    if (zz >= 0 && valid) {
+      const int64_t all_rows = (int64_t)a.n_main + a.n_bt;
+      const int64_t grow = row_off + row0 + row;
+      acc = a.zz_o + (grow * a.hq + h) * D;
+      float *accl = a.zz_lse + (int64_t)h * all_rows + grow;
+      float lnew = lse;
+      if (zz > 0) {
+        const float la = *accl;
+        const float mm = fmaxf(la, lse);
+        if (mm == kNegInf) {
+          lnew = kNegInf; wa = 0.f; wb = 0.f;
+        } else {
+          lnew = mm + logf(expf(la - mm) + expf(lse - mm));
+          wa = expf(la - lnew);
+          wb = expf(lse - lnew);
+        }
+      }
+      if (!final_out) *accl = lnew;
+      lse = lnew;
+    }
+    bf16 *og = (is_main ? a.o_m : a.o_b) + ((int64_t)(row0 + row) * a.hq + h) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      if (ok && total > 0) {
+        tmem_ld32(t_o + lane_addr + c * 32, o);
+        tc_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (!valid) continue;
+      float f[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(o[e]) * inv;
+      if (zz >= 0) {
+        float4 *ap = reinterpret_cast<float4 *>(acc + c * 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float4 prev = zz > 0 ? ap[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+          f[4 * e + 0] = wa * prev.x + wb * f[4 * e + 0];
+          f[4 * e + 1] = wa * prev.y + wb * f[4 * e + 1];
+          f[4 * e + 2] = wa * prev.z + wb * f[4 * e + 2];
+          f[4 * e + 3] = wa * prev.w + wb * f[4 * e + 3];
+          if (!final_out) ap[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+        }
+      }
+      if (final_out) {
+        uint4 *dst = reinterpret_cast<uint4 *>(og + c * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          dst[e] = make_uint4(pack_bf16(f[8 * e], f[8 * e + 1]), pack_bf16(f[8 * e + 2], f[8 * e + 3]),
+                              pack_bf16(f[8 * e + 4], f[8 * e + 5]),
+                              pack_bf16(f[8 * e + 6], f[8 * e + 7]));
+      }
+    }
+    if (valid && final_out)
+      (is_main ? a.lse_m : a.lse_b)[(int64_t)h * rows_total + row0 + row] = lse;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+bool sm100_fwd_available() { return true; }
+bool sm100_bwd_available() { return false; }
+bool sm100_available() { return true; }
+
+ba_status launch_fwd_sm100(const AttnParams &a, cudaStream_t s) {
+  TensorMaps tm;
+  const int d = a.head_dim;
+  ba_status st;
+  if ((st = make_map(&tm.q_m, a.q_m, a.n_main, a.hq, d)) != BA_OK) return st;
+  if ((st = make_map(&tm.k_m, a.k_m, a.n_main, a.hkv, d)) != BA_OK) return st;
+  if ((st = make_map(&tm.v_m, a.v_m, a.n_main, a.hkv, d)) != BA_OK) return st;
+  if (a.n_bt > 0) {
+    if ((st = make_map(&tm.q_b, a.q_b, a.n_bt, a.hq, d)) != BA_OK) return st;
+    if ((st = make_map(&tm.k_b, a.k_b, a.n_bt, a.hkv, d)) != BA_OK) return st;
+    if ((st = make_map(&tm.v_b, a.v_b, a.n_bt, a.hkv, d)) != BA_OK) return st;
+  } else {
+    tm.q_b = tm.q_m;
+    tm.k_b = tm.k_m;
+    tm.v_b = tm.v_m;
+  }
+  const int64_t grid = (int64_t)a.n_qt * a.hq;
+  if (grid == 0) return BA_OK;
+  cudaError_t e;
+  if (d == 64) {
+    const size_t smem = sizeof(FwdSmem<64>) + 1024;
+    e = cudaFuncSetAttribute(fwd_sm100_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return cuda_check(e, "fwd_sm100_kernel<64> smem");
+    fwd_sm100_kernel<64><<<(unsigned)grid, 256, smem, s>>>(a, tm);
+  } else {
+    const size_t smem = sizeof(FwdSmem<128>) + 1024;
+    e = cudaFuncSetAttribute(fwd_sm100_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return cuda_check(e, "fwd_sm100_kernel<128> smem");
+    fwd_sm100_kernel<128><<<(unsigned)grid, 256, smem, s>>>(a, tm);
+  }
+  count_launches(1);
+  return cuda_check(cudaGetLastError(), "fwd_sm100_kernel launch");
 }
 
 ba_status launch_bwd_sm100(const AttnParams &, cudaStream_t) {

@@ -75,6 +75,8 @@ ba_status launch_fwd_mma(const AttnParams &a, cudaStream_t s);
 ba_status launch_bwd_mma(const AttnParams &a, cudaStream_t s);
 // tcgen05 / TMEM / TMA kernels
 bool sm100_available();
+bool sm100_fwd_available();
+bool sm100_bwd_available();
 ba_status launch_fwd_sm100(const AttnParams &a, cudaStream_t s);
 ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s);
 
