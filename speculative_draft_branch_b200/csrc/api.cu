@@ -368,10 +368,17 @@ ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws, void *bwd_ws
   a.dq_acc = reinterpret_cast<float *>(reinterpret_cast<char *>(bwd_ws) +
                                        align_up(4 * rows * p->hq, 256));
   cudaStream_t s = (cudaStream_t)stream;
+  a.dq_out_m = (__nv_bfloat16 *)dq_m;
+  a.dq_out_b = (__nv_bfloat16 *)dq_b;
+  const bool sm100 = use_sm100_bwd();
+  // tcgen05: dK/dV and dQ kernels write every gradient directly;
+  // mma.sync: dQ is accumulated in fp32 with atomics, then converted
+  a.zero_dq_acc = sm100 ? 0 : 1;
   BA_TRY(launch_bwd_preprocess(a, s));
   record_event(1, true, s);
-  BA_TRY(use_sm100_bwd() ? launch_bwd_sm100(a, s) : launch_bwd_mma(a, s));
+  BA_TRY(sm100 ? launch_bwd_sm100(a, s) : launch_bwd_mma(a, s));
   record_event(1, false, s);
+  if (sm100) return BA_OK;
   return launch_dq_convert(a, (__nv_bfloat16 *)dq_m, (__nv_bfloat16 *)dq_b, s);
 }
 

@@ -22,22 +22,9 @@
 
 #include <mutex>
 
-#include "internal.cuh"
-#include "sm100.cuh"
+#include "attn_sm100_common.cuh"
 
 namespace ba {
-namespace {
-
-using namespace sm100;
-using bf16 = __nv_bfloat16;
-
-constexpr float kNegInf = -INFINITY;
-constexpr float kLn2 = 0.69314718055994530942f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
-
-struct TensorMaps {
-  CUtensorMap q_m, q_b, k_m, v_m, k_b, v_b;
-};
 
 // ---- host: tensor maps -------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -54,8 +41,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows, heads, d] bf16 -> 3-D map (d, heads, rows), box (64, 1, 128), 128-byte swizzle.
-ba_status make_map(CUtensorMap *m, const void *ptr, int64_t rows, int heads, int d) {
+// [rows, heads, d] bf16 -> 3-D map (d, heads, rows), box (64, 1, box_rows), 128-byte swizzle.
+ba_status make_tensor_map(CUtensorMap *m, const void *ptr, int64_t rows, int heads, int d,
+                          int box_rows) {
   auto fn = encode_fn();
   if (!fn) {
     set_error("cuTensorMapEncodeTiled unavailable");
@@ -63,7 +51,7 @@ ba_status make_map(CUtensorMap *m, const void *ptr, int64_t rows, int heads, int
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -74,6 +62,13 @@ ba_status make_map(CUtensorMap *m, const void *ptr, int64_t rows, int heads, int
   }
   return BA_OK;
 }
+
+
+namespace {
+
+using namespace sm100;
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // ---- device ---------------------------------------------------------------------
 template <int D>
@@ -87,57 +82,10 @@ struct FwdSmem {
   uint64_t bar_s_full[2], bar_s_empty[2];
   uint64_t bar_p_full[2];
   uint64_t bar_o_done;
+  uint64_t bar_o_final;  // one phase: the last PV product has landed in O
   uint32_t tmem_base;
   int abort_flag;
 };
-
-struct Seg {
-  int key0, n, kind, full_b, full_e;
-};
-
-struct TileSegs {
-  Seg s[3];
-  int total;
-  __device__ __forceinline__ void locate(int it, int &key0, int &kind, bool &full) const {
-    int si = 0, sub = it;
-    if (sub >= s[0].n) {
-      sub -= s[0].n;
-      si = 1;
-      if (sub >= s[1].n) {
-        sub -= s[1].n;
-        si = 2;
-      }
-    }
-    const Seg g = si == 0 ? s[0] : (si == 1 ? s[1] : s[2]);
-    key0 = g.key0 + sub * 128;
-    kind = g.kind;
-    full = kind == 0 && key0 >= g.full_b && key0 + 128 <= g.full_e;
-  }
-};
-
-__device__ __forceinline__ TileSegs make_segs(const AttnParams &a, int t, bool is_main) {
-  TileSegs ts;
-  int n = 0;
-  const int32_t *qt = a.plan.qtile + (int64_t)t * 6;
-  const int zz = a.zz_step;
-  if (zz < 0) {
-    const int k0 = qt[0] * 128, k1 = min(qt[3] * 128, a.n_main);
-    ts.s[n++] = {k0, (k1 - k0 + 127) / 128, 0, qt[1] * 128, qt[2] * 128};
-  } else if (zz < a.zz_C) {
-    const int32_t *z = a.plan.zz_tiles + ((int64_t)zz * a.n_qt + t) * 4;
-    for (int w = 0; w < 2; ++w) {
-      const int k0 = z[2 * w] * 128, k1 = min(z[2 * w + 1] * 128, a.n_main);
-      if (k1 > k0) ts.s[n++] = {k0, (k1 - k0 + 127) / 128, w, 0, 0};
-    }
-  }
-  if (!is_main && (zz < 0 || zz == a.zz_C)) {
-    const int b0 = qt[4], b1 = qt[5];
-    if (b1 > b0) ts.s[n++] = {b0, (b1 - b0 + 127) / 128, 2, 0, 0};
-  }
-  for (int i = n; i < 3; ++i) ts.s[i] = {0, 0, 2, 0, 0};
-  ts.total = ts.s[0].n + ts.s[1].n + ts.s[2].n;
-  return ts;
-}
 
 template <int D>
 __global__ void __launch_bounds__(256, 1)
@@ -174,6 +122,7 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(smem_u32(&sm.bar_p_full[s]), 128);
     }
     mbar_init(b_o, 1);
+    mbar_init(smem_u32(&sm.bar_o_final), 1);
     sm.abort_flag = 0;
     mbar_fence_init();
   }
@@ -264,7 +213,7 @@ __global__ void __launch_bounds__(256, 1)
         break;
       }
     }
-    if (ok && total > 0) issue_pv(total - 1);
+    if (ok && total > 0 && issue_pv(total - 1)) mma_commit(smem_u32(&sm.bar_o_final));
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
     const int row = threadIdx.x - 128;
@@ -385,8 +334,11 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.bar_p_full[sb]));
     }
+    // the epilogue may lag o_done by two phases, so it waits on its own
+    // one-phase barrier instead of a parity of o_done
     if (ok && total > 0 &&
-        !__all_sync(0xffffffffu, mbar_wait(b_o, (total - 1) & 1, abort_flag, status_word, 9)))
+        !__all_sync(0xffffffffu,
+                    mbar_wait(smem_u32(&sm.bar_o_final), 0, abort_flag, status_word, 9)))
       ok = false;
     tc_fence_after();
 
@@ -466,20 +418,19 @@ __global__ void __launch_bounds__(256, 1)
 }  // namespace
 
 bool sm100_fwd_available() { return true; }
-bool sm100_bwd_available() { return false; }
 bool sm100_available() { return true; }
 
 ba_status launch_fwd_sm100(const AttnParams &a, cudaStream_t s) {
   TensorMaps tm;
   const int d = a.head_dim;
   ba_status st;
-  if ((st = make_map(&tm.q_m, a.q_m, a.n_main, a.hq, d)) != BA_OK) return st;
-  if ((st = make_map(&tm.k_m, a.k_m, a.n_main, a.hkv, d)) != BA_OK) return st;
-  if ((st = make_map(&tm.v_m, a.v_m, a.n_main, a.hkv, d)) != BA_OK) return st;
+  if ((st = make_tensor_map(&tm.q_m, a.q_m, a.n_main, a.hq, d, 128)) != BA_OK) return st;
+  if ((st = make_tensor_map(&tm.k_m, a.k_m, a.n_main, a.hkv, d, 128)) != BA_OK) return st;
+  if ((st = make_tensor_map(&tm.v_m, a.v_m, a.n_main, a.hkv, d, 128)) != BA_OK) return st;
   if (a.n_bt > 0) {
-    if ((st = make_map(&tm.q_b, a.q_b, a.n_bt, a.hq, d)) != BA_OK) return st;
-    if ((st = make_map(&tm.k_b, a.k_b, a.n_bt, a.hkv, d)) != BA_OK) return st;
-    if ((st = make_map(&tm.v_b, a.v_b, a.n_bt, a.hkv, d)) != BA_OK) return st;
+    if ((st = make_tensor_map(&tm.q_b, a.q_b, a.n_bt, a.hq, d, 128)) != BA_OK) return st;
+    if ((st = make_tensor_map(&tm.k_b, a.k_b, a.n_bt, a.hkv, d, 128)) != BA_OK) return st;
+    if ((st = make_tensor_map(&tm.v_b, a.v_b, a.n_bt, a.hkv, d, 128)) != BA_OK) return st;
   } else {
     tm.q_b = tm.q_m;
     tm.k_b = tm.k_m;
@@ -505,9 +456,5 @@ ba_status launch_fwd_sm100(const AttnParams &a, cudaStream_t s) {
   return cuda_check(cudaGetLastError(), "fwd_sm100_kernel launch");
 }
 
-ba_status launch_bwd_sm100(const AttnParams &, cudaStream_t) {
-  set_error("tcgen05 backward kernel not built");
-  return BA_ERR_UNSUPPORTED;
-}
 
 }  // namespace ba

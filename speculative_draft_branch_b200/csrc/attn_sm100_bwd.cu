@@ -1,0 +1,668 @@
+// Backward of branch attention on the tcgen05 tensor cores (sm_100a).
+//
+// Given the merged LSE l of every query (written by the forward) and
+// D = rowsum(dO * O), every visible (query i, key k) pair has
+//   P_ik = exp(scale q_i.k_k - l_i),  dS_ik = P_ik (dO_i.v_k - D_i),
+// and the gradients are dV_k = sum_i P_ik dO_i, dK_k = scale sum_i dS_ik q_i,
+// dQ_i = scale sum_k dS_ik k_k.  P is recomputed from the merged LSE, so the
+// main-prefix and branch-local parts of a branch query share one softmax
+// normalisation, as the paper's merge rule makes them
+// ("Online Draft Co-Training", technical-contribution section).
+//
+// Two kernels, neither with atomics:
+//   dq_sm100_kernel    query-stationary (one CTA per 128-row query tile and q
+//                      head, the forward's work order): per key tile S and dP
+//                      into TMEM, dS by 256 threads (two per row), dS into
+//                      shared memory, dQ += dS K accumulated in TMEM.
+//   dkdv_sm100_kernel  key-stationary (one CTA per 128-row key tile and kv
+//                      head, the plan's backward work order): over every
+//                      64-row query chunk of every q head of the group that
+//                      visits the tile, S^T = K Q^T and dP^T = V dO^T into
+//                      (double-buffered) TMEM, P^T and dS^T into shared
+//                      memory, dV += P^T dO and dK += dS^T Q accumulated in
+//                      TMEM for the whole walk.
+#include "attn_sm100_common.cuh"
+
+namespace ba {
+namespace {
+
+using namespace sm100;
+
+// ============================================================================
+// dQ kernel
+// ============================================================================
+template <int D>
+struct DqSmem {
+  bf16 q[128 * D];
+  bf16 dout[128 * D];
+  bf16 k[2][128 * D];
+  bf16 v[2][128 * D];
+  bf16 ds[128 * 128];  // dS: two [128 rows][64 keys] halves
+  uint64_t bar_qdo;
+  uint64_t bar_kv_full[2], bar_kv_empty[2];
+  uint64_t bar_sdp_full, bar_sdp_empty;
+  uint64_t bar_ds_full, bar_ds_empty;
+  uint64_t bar_dq_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct DqMaps {
+  TensorMaps t;
+  CUtensorMap do_m, do_b;
+};
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    dq_sm100_kernel(const AttnParams a, const __grid_constant__ DqMaps tm) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  DqSmem<D> &sm = *reinterpret_cast<DqSmem<D> *>(smem_raw + (((raw + 1023) & ~1023u) - raw));
+  if (a.plan.status[0] != 0) return;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = a.plan.fwd_order[blockIdx.x / a.hq];
+  const int h = blockIdx.x % a.hq;
+  const int g = h / (a.hq / a.hkv);
+  const bool is_main = t < a.n_qt_main;
+  const int tt = is_main ? t : t - a.n_qt_main;
+  const int rows_total = is_main ? a.n_main : a.n_bt;
+  const int row0 = tt * 128;
+  const int nrows = min(128, rows_total - row0);
+  const int row_off = is_main ? 0 : a.n_main;
+  const TileSegs segs = make_segs(a, t, is_main);
+  const int total = segs.total;
+  int *status_word = a.plan.status + 1;
+  volatile int *abort_flag = &sm.abort_flag;
+
+  const uint32_t b_qdo = smem_u32(&sm.bar_qdo);
+  const uint32_t b_sdp_full = smem_u32(&sm.bar_sdp_full), b_sdp_empty = smem_u32(&sm.bar_sdp_empty);
+  const uint32_t b_ds_full = smem_u32(&sm.bar_ds_full), b_ds_empty = smem_u32(&sm.bar_ds_empty);
+  const uint32_t b_dq = smem_u32(&sm.bar_dq_done);
+  if (threadIdx.x == 0) {
+    mbar_init(b_qdo, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&sm.bar_kv_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_kv_empty[s]), 1);
+    }
+    mbar_init(b_sdp_full, 1);
+    mbar_init(b_sdp_empty, 256);
+    mbar_init(b_ds_full, 256);
+    mbar_init(b_ds_empty, 1);
+    mbar_init(b_dq, 1);
+    sm.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    if (total > 0) {
+      mbar_expect_tx(b_qdo, 2 * 128 * D * 2);
+      const CUtensorMap *qm = is_main ? &tm.t.q_m : &tm.t.q_b;
+      const CUtensorMap *dm = is_main ? &tm.do_m : &tm.do_b;
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x) {
+        tma_load_3d(smem_u32(sm.q) + x * 16384, qm, b_qdo, x * 64, h, row0);
+        tma_load_3d(smem_u32(sm.dout) + x * 16384, dm, b_qdo, x * 64, h, row0);
+      }
+    }
+    int issued = 0;
+    for (int j = 0; j < total; ++j) {
+      const int st = j & 1;
+      if (j >= 2 && !mbar_wait(smem_u32(&sm.bar_kv_empty[st]), ((j - 2) >> 1) & 1, abort_flag,
+                               status_word, 1))
+        break;
+      int key0, kind;
+      bool full;
+      segs.locate(j, key0, kind, full);
+      const CUtensorMap *km = kind == 2 ? &tm.t.k_b : &tm.t.k_m;
+      const CUtensorMap *vm = kind == 2 ? &tm.t.v_b : &tm.t.v_m;
+      const uint32_t bar = smem_u32(&sm.bar_kv_full[st]);
+      mbar_expect_tx(bar, 2 * 128 * D * 2);
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x) {
+        tma_load_3d(smem_u32(sm.k[st]) + x * 16384, km, bar, x * 64, g, key0);
+        tma_load_3d(smem_u32(sm.v[st]) + x * 16384, vm, bar, x * 64, g, key0);
+      }
+      ++issued;
+    }
+    for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
+      mbar_wait(smem_u32(&sm.bar_kv_full[j & 1]), (j >> 1) & 1, abort_flag, status_word, 2);
+    if (total > 0) mbar_wait(b_qdo, 0, abort_flag, status_word, 2);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idesc_dq = idesc_bf16(128, D, false, true);
+    bool ok = total == 0 || mbar_wait(b_qdo, 0, abort_flag, status_word, 3);
+    const uint32_t q_s = smem_u32(sm.q), do_s = smem_u32(sm.dout), ds_s = smem_u32(sm.ds);
+    auto issue_dq = [&](int i) -> bool {
+      if (!mbar_wait(b_ds_full, i & 1, abort_flag, status_word, 4)) return false;
+      tc_fence_after();
+      const uint32_t k_s = smem_u32(sm.k[i & 1]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint64_t ad = sdesc(ds_s + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc(k_s + k * 2048, 16384, 1024);
+        mma_bf16(t_dq, ad, bd, idesc_dq, (i > 0 || k > 0) ? 1u : 0u);
+      }
+      mma_commit(b_ds_empty);
+      mma_commit(smem_u32(&sm.bar_kv_empty[i & 1]));
+      mma_commit(b_dq);
+      return true;
+    };
+    for (int j = 0; ok && j < total; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(smem_u32(&sm.bar_kv_full[st]), (j >> 1) & 1, abort_flag, status_word, 5) ||
+          (j >= 1 && !mbar_wait(b_sdp_empty, (j - 1) & 1, abort_flag, status_word, 6))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t k_s = smem_u32(sm.k[st]), v_s = smem_u32(sm.v[st]);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+        mma_bf16(t_s, sdesc(q_s + off, 16, 1024), sdesc(k_s + off, 16, 1024), idesc_s,
+                 k > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+        mma_bf16(t_dp, sdesc(do_s + off, 16, 1024), sdesc(v_s + off, 16, 1024), idesc_s,
+                 k > 0 ? 1u : 0u);
+      }
+      mma_commit(b_sdp_full);
+      if (j >= 1 && !issue_dq(j - 1)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok && total > 0) issue_dq(total - 1);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ dS (2 threads / row)
+    const int ew = threadIdx.x - 128;
+    const int half = ew >> 7;
+    const int row = ew & 127;
+    const bool valid = row < nrows;
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    int lo0 = 0, hi0 = -1, lo2 = 0, hi2 = -1;
+    float lse2 = 0.f, dd = 0.f;
+    if (valid) {
+      const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[row_off + row0 + row];
+      lo0 = iv.x; hi0 = iv.y; lo2 = iv.z; hi2 = iv.w;
+      lse2 = (is_main ? a.lse_m : a.lse_b)[(int64_t)h * rows_total + row0 + row] * kLog2e;
+      dd = a.d_all[(int64_t)h * ((int64_t)a.n_main + a.n_bt) + row_off + row0 + row];
+    }
+    bool ok = true;
+    const uint32_t swz = (uint32_t)(row & 7);
+    const uint32_t ds_row = smem_u32(sm.ds) + half * 16384 + row * 128;
+    for (int j = 0; j < total; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(b_sdp_full, j & 1, abort_flag, status_word, 7))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      int key0, kind;
+      bool full;
+      segs.locate(j, key0, kind, full);
+      const int clo = kind == 2 ? lo2 : lo0, chi = kind == 2 ? hi2 : hi0;
+      float s[64], dp[64];
+      tmem_ld32(t_s + lane_addr + half * 64, reinterpret_cast<uint32_t *>(s));
+      tmem_ld32(t_s + lane_addr + half * 64 + 32, reinterpret_cast<uint32_t *>(s) + 32);
+      tmem_ld32(t_dp + lane_addr + half * 64, reinterpret_cast<uint32_t *>(dp));
+      tmem_ld32(t_dp + lane_addr + half * 64 + 32, reinterpret_cast<uint32_t *>(dp) + 32);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(b_sdp_empty);
+      const int kbase = key0 + half * 64;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const int key = kbase + c;
+        const bool vis = valid && (full || (key >= clo && key <= chi));
+        const float p = vis ? ex2(s[c] * a.scale_log2 - lse2) : 0.f;
+        dp[c] = p * (dp[c] - dd);
+      }
+      if (j >= 1 &&
+          !__all_sync(0xffffffffu, mbar_wait(b_ds_empty, (j - 1) & 1, abort_flag, status_word, 8))) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        st_shared_v4(ds_row + ((ch ^ swz) << 4), pack_bf16(dp[8 * ch], dp[8 * ch + 1]),
+                     pack_bf16(dp[8 * ch + 2], dp[8 * ch + 3]),
+                     pack_bf16(dp[8 * ch + 4], dp[8 * ch + 5]),
+                     pack_bf16(dp[8 * ch + 6], dp[8 * ch + 7]));
+      fence_proxy_async_smem();
+      mbar_arrive(b_ds_full);
+    }
+    if (ok && total > 0 &&
+        !__all_sync(0xffffffffu, mbar_wait(b_dq, (total - 1) & 1, abort_flag, status_word, 9)))
+      ok = false;
+    tc_fence_after();
+    bf16 *dst = (is_main ? a.dq_out_m : a.dq_out_b) + ((int64_t)(row0 + row) * a.hq + h) * D +
+                half * (D / 2);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      uint32_t o[32];
+      if (ok && total > 0) {
+        tmem_ld32(t_dq + lane_addr + half * (D / 2) + c * 32, o);
+        tc_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (!valid) continue;
+      uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        d4[e] = make_uint4(
+            pack_bf16(__uint_as_float(o[8 * e]) * a.scale, __uint_as_float(o[8 * e + 1]) * a.scale),
+            pack_bf16(__uint_as_float(o[8 * e + 2]) * a.scale,
+                      __uint_as_float(o[8 * e + 3]) * a.scale),
+            pack_bf16(__uint_as_float(o[8 * e + 4]) * a.scale,
+                      __uint_as_float(o[8 * e + 5]) * a.scale),
+            pack_bf16(__uint_as_float(o[8 * e + 6]) * a.scale,
+                      __uint_as_float(o[8 * e + 7]) * a.scale));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================
+// dK / dV kernel
+// ============================================================================
+constexpr int kQc = 64;  // query rows per chunk
+
+template <int D>
+struct DkvSmem {
+  bf16 k[128 * D];
+  bf16 v[128 * D];
+  bf16 q[2][kQc * D];        // D/64 boxes of [64 rows][64], 8 KB each
+  bf16 dout[2][kQc * D];
+  bf16 pt[2][128 * kQc];     // P^T  [128 keys][64 queries]
+  bf16 dst[2][128 * kQc];    // dS^T [128 keys][64 queries]
+  float lse2[2][kQc];        // LSE of each query, log2 units
+  float dd[2][kQc];          // D of each query
+  int lo[2][kQc], hi[2][kQc];  // key interval of each query (empty: lo > hi)
+  uint64_t bar_kv;
+  uint64_t bar_qdo_full[2], bar_qdo_empty[2], bar_vec_full[2];
+  uint64_t bar_sdp_full[2], bar_sdp_empty[2];
+  uint64_t bar_pds_full[2], bar_pds_empty[2];
+  uint64_t bar_acc_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct DkvMaps {
+  TensorMaps t;
+  CUtensorMap q64_m, q64_b, do64_m, do64_b;  // 64-row boxes
+};
+
+struct ChunkWalk {
+  int n_t0, n_t1, t0, t1, per_head, grp, g;
+  __device__ __forceinline__ void at(int c, const AttnParams &a, int &h, bool &is_main_q,
+                                     int &tile, int &row0, int &nrows) const {
+    const int hh = c / per_head, rem = c % per_head;
+    const int ti = rem >> 1, half = rem & 1;
+    h = g * grp + hh;
+    is_main_q = ti < n_t0;
+    tile = is_main_q ? t0 + ti : t1 + (ti - n_t0);
+    const int rows = is_main_q ? a.n_main : a.n_bt;
+    row0 = tile * 128 + half * kQc;
+    nrows = max(0, min(kQc, rows - row0));
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    dkdv_sm100_kernel(const AttnParams a, const __grid_constant__ DkvMaps tm) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  DkvSmem<D> &sm = *reinterpret_cast<DkvSmem<D> *>(smem_raw + (((raw + 1023) & ~1023u) - raw));
+  if (a.plan.status[0] != 0) return;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int item = a.plan.bwd_order[blockIdx.x / a.hkv];
+  const int g = blockIdx.x % a.hkv;
+  const bool main_kv = item < a.n_kt;
+  const int kt = main_kv ? item : item - a.n_kt;
+  const int key0 = kt * 128;
+  const int n_keys = main_kv ? a.n_main : a.n_bt;
+  ChunkWalk cw;
+  cw.grp = a.hq / a.hkv;
+  cw.g = g;
+  if (main_kv) {
+    const int32_t *r = a.plan.kv_main + (int64_t)kt * 4;
+    cw.t0 = r[0]; cw.n_t0 = r[1] - r[0]; cw.t1 = r[2]; cw.n_t1 = r[3] - r[2];
+  } else {
+    const int32_t *r = a.plan.kv_branch + (int64_t)kt * 2;
+    cw.t0 = 0; cw.n_t0 = 0; cw.t1 = r[0]; cw.n_t1 = r[1] - r[0];
+  }
+  cw.per_head = 2 * (cw.n_t0 + cw.n_t1);
+  const int total = cw.grp * cw.per_head;
+  int *status_word = a.plan.status + 1;
+  volatile int *abort_flag = &sm.abort_flag;
+  const int64_t all_rows = (int64_t)a.n_main + a.n_bt;
+
+  const uint32_t b_kv = smem_u32(&sm.bar_kv), b_acc = smem_u32(&sm.bar_acc_done);
+  if (threadIdx.x == 0) {
+    mbar_init(b_kv, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&sm.bar_qdo_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_qdo_empty[s]), 1);
+      mbar_init(smem_u32(&sm.bar_vec_full[s]), 32);
+      mbar_init(smem_u32(&sm.bar_sdp_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_sdp_empty[s]), 128);
+      mbar_init(smem_u32(&sm.bar_pds_full[s]), 128);
+      mbar_init(smem_u32(&sm.bar_pds_empty[s]), 1);
+    }
+    mbar_init(b_acc, 1);
+    sm.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t t_dk = tmem, t_dv = tmem + 128;
+  auto t_s = [&](int b) { return tmem + 256 + b * 64; };
+  auto t_dp = [&](int b) { return tmem + 384 + b * 64; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // lane 0 issues the TMA tile loads, all lanes stage the per-query vectors
+    if (lane == 0 && total > 0) {
+      mbar_expect_tx(b_kv, 2 * 128 * D * 2);
+      const CUtensorMap *km = main_kv ? &tm.t.k_m : &tm.t.k_b;
+      const CUtensorMap *vm = main_kv ? &tm.t.v_m : &tm.t.v_b;
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x) {
+        tma_load_3d(smem_u32(sm.k) + x * 16384, km, b_kv, x * 64, g, key0);
+        tma_load_3d(smem_u32(sm.v) + x * 16384, vm, b_kv, x * 64, g, key0);
+      }
+    }
+    int issued = 0;
+    for (int c = 0; c < total; ++c) {
+      const int st = c & 1;
+      if (c >= 2 && !__all_sync(0xffffffffu,
+                                mbar_wait(smem_u32(&sm.bar_qdo_empty[st]), ((c - 2) >> 1) & 1,
+                                          abort_flag, status_word, 1)))
+        break;
+      int h, tile, row0, nrows;
+      bool is_main_q;
+      cw.at(c, a, h, is_main_q, tile, row0, nrows);
+      if (lane == 0) {
+        const uint32_t bar = smem_u32(&sm.bar_qdo_full[st]);
+        mbar_expect_tx(bar, 2 * kQc * D * 2);
+        const CUtensorMap *qm = is_main_q ? &tm.q64_m : &tm.q64_b;
+        const CUtensorMap *dm = is_main_q ? &tm.do64_m : &tm.do64_b;
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x) {
+          tma_load_3d(smem_u32(sm.q[st]) + x * 8192, qm, bar, x * 64, h, row0);
+          tma_load_3d(smem_u32(sm.dout[st]) + x * 8192, dm, bar, x * 64, h, row0);
+        }
+      }
+      const int rows = is_main_q ? a.n_main : a.n_bt;
+      const int roff = is_main_q ? 0 : a.n_main;
+      const float *lse = is_main_q ? a.lse_m : a.lse_b;
+#pragma unroll
+      for (int i = 0; i < kQc / 32; ++i) {
+        const int r = lane + 32 * i;
+        float l2 = 0.f, dv = 0.f;
+        int lo = 1, hi = 0;
+        if (r < nrows) {
+          l2 = lse[(int64_t)h * rows + row0 + r] * kLog2e;
+          dv = a.d_all[(int64_t)h * all_rows + roff + row0 + r];
+          const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[roff + row0 + r];
+          lo = main_kv ? iv.x : iv.z;
+          hi = main_kv ? iv.y : iv.w;
+        }
+        sm.lse2[st][r] = l2;
+        sm.dd[st][r] = dv;
+        sm.lo[st][r] = lo;
+        sm.hi[st][r] = hi;
+      }
+      mbar_arrive(smem_u32(&sm.bar_vec_full[st]));
+      ++issued;
+    }
+    if (lane == 0) {
+      for (int c = (issued > 2 ? issued - 2 : 0); c < issued; ++c)
+        mbar_wait(smem_u32(&sm.bar_qdo_full[c & 1]), (c >> 1) & 1, abort_flag, status_word, 2);
+      if (total > 0) mbar_wait(b_kv, 0, abort_flag, status_word, 2);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_s = idesc_bf16(128, kQc, false, false);
+    constexpr uint32_t idesc_g = idesc_bf16(128, D, false, true);
+    bool ok = total == 0 || mbar_wait(b_kv, 0, abort_flag, status_word, 3);
+    const uint32_t k_s = smem_u32(sm.k), v_s = smem_u32(sm.v);
+    auto grads = [&](int i) -> bool {
+      const int sb = i & 1;
+      if (!mbar_wait(smem_u32(&sm.bar_pds_full[sb]), (i >> 1) & 1, abort_flag, status_word, 4))
+        return false;
+      tc_fence_after();
+      const uint32_t p_s = smem_u32(sm.pt[sb]), ds_s = smem_u32(sm.dst[sb]);
+      const uint32_t q_s = smem_u32(sm.q[sb]), do_s = smem_u32(sm.dout[sb]);
+#pragma unroll
+      for (int k = 0; k < kQc / 16; ++k)
+        mma_bf16(t_dv, sdesc(p_s + k * 32, 16, 1024), sdesc(do_s + k * 2048, 8192, 1024), idesc_g,
+                 (i > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+      for (int k = 0; k < kQc / 16; ++k)
+        mma_bf16(t_dk, sdesc(ds_s + k * 32, 16, 1024), sdesc(q_s + k * 2048, 8192, 1024), idesc_g,
+                 (i > 0 || k > 0) ? 1u : 0u);
+      mma_commit(smem_u32(&sm.bar_pds_empty[sb]));
+      mma_commit(smem_u32(&sm.bar_qdo_empty[sb]));
+      return true;
+    };
+    for (int c = 0; ok && c < total; ++c) {
+      const int st = c & 1;
+      if (!mbar_wait(smem_u32(&sm.bar_qdo_full[st]), (c >> 1) & 1, abort_flag, status_word, 5) ||
+          (c >= 2 && !mbar_wait(smem_u32(&sm.bar_sdp_empty[st]), ((c - 2) >> 1) & 1, abort_flag,
+                                status_word, 6))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t q_s = smem_u32(sm.q[st]), do_s = smem_u32(sm.dout[st]);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
+        const uint32_t qa = (k >> 2) * 8192 + (k & 3) * 32;
+        mma_bf16(t_s(st), sdesc(k_s + ka, 16, 1024), sdesc(q_s + qa, 16, 1024), idesc_s,
+                 k > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
+        const uint32_t qa = (k >> 2) * 8192 + (k & 3) * 32;
+        mma_bf16(t_dp(st), sdesc(v_s + ka, 16, 1024), sdesc(do_s + qa, 16, 1024), idesc_s,
+                 k > 0 ? 1u : 0u);
+      }
+      mma_commit(smem_u32(&sm.bar_sdp_full[st]));
+      if (c >= 1 && !grads(c - 1)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok && total > 0 && grads(total - 1)) mma_commit(b_acc);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ P^T, dS^T (1 thread / key)
+    const int row = threadIdx.x - 128;
+    const int key = key0 + row;
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t swz = (uint32_t)(row & 7);
+    bool ok = true;
+    for (int c = 0; c < total; ++c) {
+      const int st = c & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_sdp_full[st]), (c >> 1) & 1,
+                                             abort_flag, status_word, 7))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[kQc], dp[kQc];
+      tmem_ld32(t_s(st) + lane_addr, reinterpret_cast<uint32_t *>(s));
+      tmem_ld32(t_s(st) + lane_addr + 32, reinterpret_cast<uint32_t *>(s) + 32);
+      tmem_ld32(t_dp(st) + lane_addr, reinterpret_cast<uint32_t *>(dp));
+      tmem_ld32(t_dp(st) + lane_addr + 32, reinterpret_cast<uint32_t *>(dp) + 32);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.bar_sdp_empty[st]));
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_vec_full[st]), (c >> 1) & 1,
+                                             abort_flag, status_word, 8))) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int q = 0; q < kQc; ++q) {
+        const bool vis = key >= sm.lo[st][q] && key <= sm.hi[st][q];
+        const float p = vis ? ex2(s[q] * a.scale_log2 - sm.lse2[st][q]) : 0.f;
+        s[q] = p;
+        dp[q] = p * (dp[q] - sm.dd[st][q]);
+      }
+      if (c >= 2 && !__all_sync(0xffffffffu,
+                                mbar_wait(smem_u32(&sm.bar_pds_empty[st]), ((c - 2) >> 1) & 1,
+                                          abort_flag, status_word, 9))) {
+        ok = false;
+        break;
+      }
+      const uint32_t p_row = smem_u32(sm.pt[st]) + row * 128;
+      const uint32_t d_row = smem_u32(sm.dst[st]) + row * 128;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        st_shared_v4(p_row + ((ch ^ swz) << 4), pack_bf16(s[8 * ch], s[8 * ch + 1]),
+                     pack_bf16(s[8 * ch + 2], s[8 * ch + 3]), pack_bf16(s[8 * ch + 4], s[8 * ch + 5]),
+                     pack_bf16(s[8 * ch + 6], s[8 * ch + 7]));
+        st_shared_v4(d_row + ((ch ^ swz) << 4), pack_bf16(dp[8 * ch], dp[8 * ch + 1]),
+                     pack_bf16(dp[8 * ch + 2], dp[8 * ch + 3]),
+                     pack_bf16(dp[8 * ch + 4], dp[8 * ch + 5]),
+                     pack_bf16(dp[8 * ch + 6], dp[8 * ch + 7]));
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&sm.bar_pds_full[st]));
+    }
+    if (ok && total > 0 &&
+        !__all_sync(0xffffffffu, mbar_wait(b_acc, 0, abort_flag, status_word, 10)))
+      ok = false;
+    tc_fence_after();
+    const bool valid = key < n_keys;
+    bf16 *dkg = (main_kv ? a.dk_m : a.dk_b) + ((int64_t)key * a.hkv + g) * D;
+    bf16 *dvg = (main_kv ? a.dv_m : a.dv_b) + ((int64_t)key * a.hkv + g) * D;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      const uint32_t src = part == 0 ? t_dk : t_dv;
+      const float mul = part == 0 ? a.scale : 1.f;
+      bf16 *dst = part == 0 ? dkg : dvg;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (ok && total > 0) {
+          tmem_ld32(src + lane_addr + c * 32, o);
+          tc_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        if (!valid) continue;
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          d4[e] = make_uint4(
+              pack_bf16(__uint_as_float(o[8 * e]) * mul, __uint_as_float(o[8 * e + 1]) * mul),
+              pack_bf16(__uint_as_float(o[8 * e + 2]) * mul, __uint_as_float(o[8 * e + 3]) * mul),
+              pack_bf16(__uint_as_float(o[8 * e + 4]) * mul, __uint_as_float(o[8 * e + 5]) * mul),
+              pack_bf16(__uint_as_float(o[8 * e + 6]) * mul, __uint_as_float(o[8 * e + 7]) * mul));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+template <typename K, typename M>
+ba_status launch_kernel(K kernel, size_t smem, int64_t grid, int threads, const AttnParams &a,
+                        const M &maps, cudaStream_t s, const char *name) {
+  if (grid <= 0) return BA_OK;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_check(e, name);
+  kernel<<<(unsigned)grid, threads, smem, s>>>(a, maps);
+  count_launches(1);
+  return cuda_check(cudaGetLastError(), name);
+}
+
+}  // namespace
+
+bool sm100_bwd_available() { return true; }
+
+ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s) {
+  const int d = a.head_dim;
+  TensorMaps t;
+  ba_status st;
+  const bool br = a.n_bt > 0;
+#define BA_MAP(dst, ptr, rows, heads, box)                                      \
+  if ((st = make_tensor_map(&(dst), ptr, rows, heads, d, box)) != BA_OK) return st;
+  BA_MAP(t.q_m, a.q_m, a.n_main, a.hq, 128)
+  BA_MAP(t.k_m, a.k_m, a.n_main, a.hkv, 128)
+  BA_MAP(t.v_m, a.v_m, a.n_main, a.hkv, 128)
+  if (br) {
+    BA_MAP(t.q_b, a.q_b, a.n_bt, a.hq, 128)
+    BA_MAP(t.k_b, a.k_b, a.n_bt, a.hkv, 128)
+    BA_MAP(t.v_b, a.v_b, a.n_bt, a.hkv, 128)
+  } else {
+    t.q_b = t.q_m; t.k_b = t.k_m; t.v_b = t.v_m;
+  }
+  DqMaps dqm;
+  dqm.t = t;
+  BA_MAP(dqm.do_m, a.do_m, a.n_main, a.hq, 128)
+  if (br) { BA_MAP(dqm.do_b, a.do_b, a.n_bt, a.hq, 128) } else { dqm.do_b = dqm.do_m; }
+  DkvMaps kvm;
+  kvm.t = t;
+  BA_MAP(kvm.q64_m, a.q_m, a.n_main, a.hq, kQc)
+  BA_MAP(kvm.do64_m, a.do_m, a.n_main, a.hq, kQc)
+  if (br) {
+    BA_MAP(kvm.q64_b, a.q_b, a.n_bt, a.hq, kQc)
+    BA_MAP(kvm.do64_b, a.do_b, a.n_bt, a.hq, kQc)
+  } else {
+    kvm.q64_b = kvm.q64_m; kvm.do64_b = kvm.do64_m;
+  }
+#undef BA_MAP
+  const int64_t grid_dq = (int64_t)a.n_qt * a.hq;
+  const int64_t grid_kv = (int64_t)(a.n_kt + a.n_bkt) * a.hkv;
+  if (d == 64) {
+    if ((st = launch_kernel(dkdv_sm100_kernel<64>, sizeof(DkvSmem<64>) + 1024, grid_kv, 256, a,
+                            kvm, s, "dkdv_sm100_kernel<64>")) != BA_OK)
+      return st;
+    return launch_kernel(dq_sm100_kernel<64>, sizeof(DqSmem<64>) + 1024, grid_dq, 384, a, dqm, s,
+                         "dq_sm100_kernel<64>");
+  }
+  if ((st = launch_kernel(dkdv_sm100_kernel<128>, sizeof(DkvSmem<128>) + 1024, grid_kv, 256, a,
+                          kvm, s, "dkdv_sm100_kernel<128>")) != BA_OK)
+    return st;
+  return launch_kernel(dq_sm100_kernel<128>, sizeof(DqSmem<128>) + 1024, grid_dq, 384, a, dqm, s,
+                       "dq_sm100_kernel<128>");
+}
+
+}  // namespace ba

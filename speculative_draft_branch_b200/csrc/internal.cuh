@@ -39,6 +39,8 @@ struct AttnParams {
   const float *d_all;         // D [Hq, N + Nb]
   float *dq_acc;              // [(N + Nb), Hq, d] fp32
   __nv_bfloat16 *dk_m, *dv_m, *dk_b, *dv_b;
+  __nv_bfloat16 *dq_out_m, *dq_out_b;  // dQ written directly (tcgen05 backward)
+  int32_t zero_dq_acc;                  // preprocess clears dq_acc (mma.sync backward)
   // zigzag partial output (fp32 O accumulator [(N+Nb), Hq, d], LSE [Hq, N+Nb])
   float *zz_o;
   float *zz_lse;

@@ -96,8 +96,8 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, int heads,
 
 // ---- backward preprocess ---------------------------------------------------
 // D[h, row] = sum_d dO[row, h, d] * O[row, h, d] (fp32 accumulate), rows =
-// main rows then branch rows; the fp32 dQ accumulator of the same row-head is
-// zeroed in the same pass.
+// main rows then branch rows; when the backward accumulates dQ with atomics
+// the fp32 dQ accumulator of the same row-head is zeroed in the same pass.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(AttnParams a) {
   constexpr int kLanes = D / 8;
@@ -127,9 +127,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(AttnParams a) {
       unpack8(*reinterpret_cast<const uint4 *>(dout + off), y);
 #pragma unroll
       for (int i = 0; i < 8; ++i) s += x[i] * y[i];
-      float4 *dq = reinterpret_cast<float4 *>(a.dq_acc + (row * a.hq + h) * D + lane * 8);
-      dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.zero_dq_acc) {
+        float4 *dq = reinterpret_cast<float4 *>(a.dq_acc + (row * a.hq + h) * D + lane * 8);
+        dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
 #pragma unroll
     for (int o2 = kLanes / 2; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
