@@ -157,9 +157,17 @@ size_t fwd_ws_bytes(const ba_problem &p) {
   return align_up(4 * rows * p.hq * p.head_dim, 256) + align_up(4 * rows * p.hq, 256);
 }
 
+size_t rows_padded(const ba_problem &p) {
+  return align_up((size_t)p.n_main, 128) + align_up((size_t)p.n_branch_tokens, 128);
+}
+
+// D [Hq, rows] fp32, then one region used either as the fp32 dQ accumulator
+// (mma.sync backward) or as the per-query records (tcgen05 backward).
 size_t bwd_ws_bytes(const ba_problem &p) {
   const size_t rows = (size_t)p.n_main + p.n_branch_tokens;
-  return align_up(4 * rows * p.hq, 256) + align_up(4 * rows * p.hq * p.head_dim, 256);
+  const size_t acc = 4 * rows * p.hq * p.head_dim;
+  const size_t rec = 2 * 16 * rows_padded(p) * p.hq;
+  return align_up(4 * rows * p.hq, 256) + align_up(acc > rec ? acc : rec, 256);
 }
 
 AttnParams make_params(const ba_problem &p, const ba_plan_layout &L, const void *plan_ws) {
@@ -374,6 +382,11 @@ ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws, void *bwd_ws
   // tcgen05: dK/dV and dQ kernels write every gradient directly;
   // mma.sync: dQ is accumulated in fp32 with atomics, then converted
   a.zero_dq_acc = sm100 ? 0 : 1;
+  if (sm100) {
+    a.rec = reinterpret_cast<float4 *>(a.dq_acc);
+    a.n_main_pad = (int32_t)align_up((size_t)p->n_main, 128);
+    a.rows_pad = (int32_t)rows_padded(*p);
+  }
   BA_TRY(launch_bwd_preprocess(a, s));
   record_event(1, true, s);
   BA_TRY(sm100 ? launch_bwd_sm100(a, s) : launch_bwd_mma(a, s));

@@ -1,16 +1,16 @@
 // Branch attention on the 5th-generation tensor cores (tcgen05, sm_100a).
 //
 // Forward kernel: one CTA per (query tile of 128 rows, q head), 8 warps.
-//   warp 0      TMA producer: Q once, then a 2-stage ring of 128-key K/V tiles
+//   warp 0      TMA producer: Q once, then 3-stage rings of 128-key K tiles
+//               and V tiles (K is refilled as soon as S has read it)
 //   warp 1      MMA issuer (one thread): S_j = Q K_j^T into TMEM (two S
 //               buffers, so S_{j+1} runs while tile j is in softmax), then
-//               O += P_j V_j with O accumulating in TMEM
-//   warp 2      TMEM allocation (512 columns: S0, S1, O)
+//               O += P_j V_j with P read from TMEM and O accumulating there
+//   warp 2      TMEM allocation (512 columns: S0, S1, O, P0, P1)
 //   warps 4-7   softmax, one thread per query row (= TMEM lane): reads its S
 //               row, masks it with the row's key interval, keeps the running
-//               max / sum, writes P (bf16) into shared memory in the 128-byte
-//               swizzled K-major layout the MMA reads, and rescales its O row
-//               in TMEM only when the running max grew by more than 2^8.
+//               max / sum, writes P (bf16 pairs) back to TMEM, and rescales
+//               its O row only when the running max grew by more than 2^8.
 // Key tiles come from the plan: the main key tiles of the query tile, then
 // (branch tiles) the branch-local key rows.  Folding each tile's partial into
 // the running (O, l) is the online-softmax merge; the branch-local tiles come
@@ -71,14 +71,16 @@ using namespace sm100;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // ---- device ---------------------------------------------------------------------
+constexpr int kFwdStages = 3;
+
 template <int D>
 struct FwdSmem {
-  bf16 q[128 * D];        // D/64 boxes of [128 rows][64], 16 KB each
-  bf16 k[2][128 * D];
-  bf16 v[2][128 * D];
-  bf16 p[2][128 * 128];   // P: two [128 rows][64 keys] halves
+  bf16 q[128 * D];              // D/64 boxes of [128 rows][64], 16 KB each
+  bf16 k[kFwdStages][128 * D];
+  bf16 v[kFwdStages][128 * D];
   uint64_t bar_q;
-  uint64_t bar_kv_full[2], bar_kv_empty[2];
+  uint64_t bar_k_full[kFwdStages], bar_k_empty[kFwdStages];
+  uint64_t bar_v_full[kFwdStages], bar_v_empty[kFwdStages];
   uint64_t bar_s_full[2], bar_s_empty[2];
   uint64_t bar_p_full[2];
   uint64_t bar_o_done;
@@ -87,6 +89,8 @@ struct FwdSmem {
   int abort_flag;
 };
 
+// TMEM columns: S double-buffered at 0 and 128, O at 256, P (bf16 pairs)
+// double-buffered at 384 and 448.
 template <int D>
 __global__ void __launch_bounds__(256, 1)
     fwd_sm100_kernel(const AttnParams a, const __grid_constant__ TensorMaps tm) {
@@ -112,17 +116,22 @@ __global__ void __launch_bounds__(256, 1)
   volatile int *abort_flag = &sm.abort_flag;
 
   const uint32_t b_q = smem_u32(&sm.bar_q), b_o = smem_u32(&sm.bar_o_done);
+  const uint32_t b_final = smem_u32(&sm.bar_o_final);
   if (threadIdx.x == 0) {
     mbar_init(b_q, 1);
+    for (int s = 0; s < kFwdStages; ++s) {
+      mbar_init(smem_u32(&sm.bar_k_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_k_empty[s]), 1);
+      mbar_init(smem_u32(&sm.bar_v_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_v_empty[s]), 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&sm.bar_kv_full[s]), 1);
-      mbar_init(smem_u32(&sm.bar_kv_empty[s]), 1);
       mbar_init(smem_u32(&sm.bar_s_full[s]), 1);
       mbar_init(smem_u32(&sm.bar_s_empty[s]), 128);
       mbar_init(smem_u32(&sm.bar_p_full[s]), 128);
     }
     mbar_init(b_o, 1);
-    mbar_init(smem_u32(&sm.bar_o_final), 1);
+    mbar_init(b_final, 1);
     sm.abort_flag = 0;
     mbar_fence_init();
   }
@@ -135,6 +144,7 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const uint32_t t_o = tmem + 256;
+  auto t_p = [&](int b) { return tmem + 384 + b * 64; };
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -145,29 +155,41 @@ __global__ void __launch_bounds__(256, 1)
       for (int x = 0; x < D / 64; ++x)
         tma_load_3d(smem_u32(sm.q) + x * 16384, qmap, b_q, x * 64, h, row0);
     }
-    int issued = 0;
+    int issued_k = 0, issued_v = 0;
     for (int j = 0; j < total; ++j) {
-      const int st = j & 1;
-      if (j >= 2 && !mbar_wait(smem_u32(&sm.bar_kv_empty[st]), ((j - 2) >> 1) & 1, abort_flag,
-                               status_word, 1))
-        break;
+      const int st = j % kFwdStages;
+      const uint32_t ph = ((j / kFwdStages) - 1) & 1;
       int key0, kind;
       bool full;
       segs.locate(j, key0, kind, full);
-      const CUtensorMap *km = kind == 2 ? &tm.k_b : &tm.k_m;
-      const CUtensorMap *vm = kind == 2 ? &tm.v_b : &tm.v_m;
-      const uint32_t bar = smem_u32(&sm.bar_kv_full[st]);
-      mbar_expect_tx(bar, 2 * 128 * D * 2);
+      if (j >= kFwdStages &&
+          !mbar_wait(smem_u32(&sm.bar_k_empty[st]), ph, abort_flag, status_word, 1))
+        break;
+      const uint32_t kb = smem_u32(&sm.bar_k_full[st]);
+      mbar_expect_tx(kb, 128 * D * 2);
 #pragma unroll
-      for (int x = 0; x < D / 64; ++x) {
-        tma_load_3d(smem_u32(sm.k[st]) + x * 16384, km, bar, x * 64, g, key0);
-        tma_load_3d(smem_u32(sm.v[st]) + x * 16384, vm, bar, x * 64, g, key0);
-      }
-      ++issued;
+      for (int x = 0; x < D / 64; ++x)
+        tma_load_3d(smem_u32(sm.k[st]) + x * 16384, kind == 2 ? &tm.k_b : &tm.k_m, kb, x * 64, g,
+                    key0);
+      ++issued_k;
+      if (j >= kFwdStages &&
+          !mbar_wait(smem_u32(&sm.bar_v_empty[st]), ph, abort_flag, status_word, 1))
+        break;
+      const uint32_t vb = smem_u32(&sm.bar_v_full[st]);
+      mbar_expect_tx(vb, 128 * D * 2);
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x)
+        tma_load_3d(smem_u32(sm.v[st]) + x * 16384, kind == 2 ? &tm.v_b : &tm.v_m, vb, x * 64, g,
+                    key0);
+      ++issued_v;
     }
     // on abort: let the loads already issued land before the CTA exits
-    for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-      mbar_wait(smem_u32(&sm.bar_kv_full[j & 1]), (j >> 1) & 1, abort_flag, status_word, 2);
+    for (int j = (issued_k > kFwdStages ? issued_k - kFwdStages : 0); j < issued_k; ++j)
+      mbar_wait(smem_u32(&sm.bar_k_full[j % kFwdStages]), (j / kFwdStages) & 1, abort_flag,
+                status_word, 2);
+    for (int j = (issued_v > kFwdStages ? issued_v - kFwdStages : 0); j < issued_v; ++j)
+      mbar_wait(smem_u32(&sm.bar_v_full[j % kFwdStages]), (j / kFwdStages) & 1, abort_flag,
+                status_word, 2);
     if (total > 0) mbar_wait(b_q, 0, abort_flag, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
@@ -176,25 +198,27 @@ __global__ void __launch_bounds__(256, 1)
     bool ok = total == 0 || mbar_wait(b_q, 0, abort_flag, status_word, 3);
     const uint32_t q_s = smem_u32(sm.q);
     auto issue_pv = [&](int i) -> bool {
-      const int pb = i & 1;
-      if (!mbar_wait(smem_u32(&sm.bar_p_full[pb]), (i >> 1) & 1, abort_flag, status_word, 4))
+      const int pb = i & 1, st = i % kFwdStages;
+      if (!mbar_wait(smem_u32(&sm.bar_v_full[st]), (i / kFwdStages) & 1, abort_flag, status_word,
+                     4) ||
+          !mbar_wait(smem_u32(&sm.bar_p_full[pb]), (i >> 1) & 1, abort_flag, status_word, 4))
         return false;
       tc_fence_after();
-      const uint32_t p_s = smem_u32(sm.p[pb]), v_s = smem_u32(sm.v[pb]);
+      const uint32_t v_s = smem_u32(sm.v[st]);
+      // O += P V: P (bf16 pairs) from TMEM, V as an MN-major operand
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint64_t ad = sdesc(p_s + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-        const uint64_t bd = sdesc(v_s + k * 2048, 16384, 1024);
-        mma_bf16(t_o, ad, bd, idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
-      }
+      for (int k = 0; k < 8; ++k)
+        mma_bf16_ts(t_o, t_p(pb) + k * 8, sdesc(v_s + k * 2048, 16384, 1024), idesc_pv,
+                    (i > 0 || k > 0) ? 1u : 0u);
       mma_commit(b_o);
-      mma_commit(smem_u32(&sm.bar_kv_empty[pb]));
+      mma_commit(smem_u32(&sm.bar_v_empty[st]));
       return true;
     };
     for (int j = 0; ok && j < total; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(smem_u32(&sm.bar_kv_full[st]), (j >> 1) & 1, abort_flag, status_word, 5) ||
-          (j >= 2 && !mbar_wait(smem_u32(&sm.bar_s_empty[st]), ((j - 2) >> 1) & 1, abort_flag,
+      const int st = j % kFwdStages, sb = j & 1;
+      if (!mbar_wait(smem_u32(&sm.bar_k_full[st]), (j / kFwdStages) & 1, abort_flag, status_word,
+                     5) ||
+          (j >= 2 && !mbar_wait(smem_u32(&sm.bar_s_empty[sb]), ((j - 2) >> 1) & 1, abort_flag,
                                 status_word, 6))) {
         ok = false;
         break;
@@ -204,16 +228,17 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-        mma_bf16(tmem + st * 128, sdesc(q_s + off, 16, 1024), sdesc(k_s + off, 16, 1024),
+        mma_bf16(tmem + sb * 128, sdesc(q_s + off, 16, 1024), sdesc(k_s + off, 16, 1024),
                  idesc_qk, k > 0 ? 1u : 0u);
       }
-      mma_commit(smem_u32(&sm.bar_s_full[st]));
+      mma_commit(smem_u32(&sm.bar_s_full[sb]));
+      mma_commit(smem_u32(&sm.bar_k_empty[st]));
       if (j >= 1 && !issue_pv(j - 1)) {
         ok = false;
         break;
       }
     }
-    if (ok && total > 0 && issue_pv(total - 1)) mma_commit(smem_u32(&sm.bar_o_final));
+    if (ok && total > 0 && issue_pv(total - 1)) mma_commit(b_final);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
     const int row = threadIdx.x - 128;
@@ -247,10 +272,10 @@ __global__ void __launch_bounds__(256, 1)
         }
       }
     }
+    // running max (log2 units, possibly stale by < 2^8) and sum
     float m_used = kNegInf, l = 0.f;
     bool ok = true;
-    const uint32_t p_row = row * 128;
-    const uint32_t swz = (uint32_t)(row & 7);
+    const float sl2 = a.scale_log2;
     for (int j = 0; j < total; ++j) {
       const int sb = j & 1;
       // warp-uniform decisions: tcgen05.ld / st below are warp-collective
@@ -272,21 +297,21 @@ __global__ void __launch_bounds__(256, 1)
       tc_wait_ld();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.bar_s_empty[sb]));
-      float mx = kNegInf;
-      if (full && valid) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          s[c] *= a.scale_log2;
-          mx = fmaxf(mx, s[c]);
-        }
-      } else {
+      // mask (raw scores; the positive scale is applied after the max)
+      if (!(full && valid)) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
           const int key = key0 + c;
-          s[c] = (key >= clo && key <= chi) ? s[c] * a.scale_log2 : kNegInf;
-          mx = fmaxf(mx, s[c]);
+          if (key < clo || key > chi) s[c] = kNegInf;
         }
       }
+      float mx4[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+#pragma unroll
+      for (int c = 0; c < 128; c += 4) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx4[e] = fmaxf(mx4[e], s[c + e]);
+      }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
       const float m_new = fmaxf(m_used, mx);
       const bool need = m_new > m_used + kRescaleThreshold;
       const float alpha = need ? ex2(m_used - m_new) : 1.f;
@@ -314,31 +339,32 @@ __global__ void __launch_bounds__(256, 1)
         m_used = m_new;
       }
       const float msub = m_used == kNegInf ? 0.f : m_used;
-      const uint32_t p_s = smem_u32(sm.p[sb]);
+      // P = 2^(scale log2(e) s - m), packed to bf16 pairs in place
+      uint32_t *pk = reinterpret_cast<uint32_t *>(s);
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int c = 0; c < 128; c += 4) {
+        float pv[4];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          float pv[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            pv[e] = ex2(s[half * 64 + ch * 8 + e] - msub);
-            l += pv[e];
-          }
-          st_shared_v4(p_s + half * 16384 + p_row + ((ch ^ swz) << 4), pack_bf16(pv[0], pv[1]),
-                       pack_bf16(pv[2], pv[3]), pack_bf16(pv[4], pv[5]),
-                       pack_bf16(pv[6], pv[7]));
+        for (int e = 0; e < 4; ++e) {
+          pv[e] = ex2(fmaf(s[c + e], sl2, -msub));
+          l4[e] += pv[e];
         }
+        pk[c / 2] = pack_bf16(pv[0], pv[1]);
+        pk[c / 2 + 1] = pack_bf16(pv[2], pv[3]);
       }
-      fence_proxy_async_smem();
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      // P buffer sb was last read by PV_{j-2}, which completed before S_j
+      tmem_st32(t_p(sb) + lane_addr, pk);
+      tmem_st32(t_p(sb) + lane_addr + 32, pk + 32);
+      tc_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.bar_p_full[sb]));
     }
     // the epilogue may lag o_done by two phases, so it waits on its own
     // one-phase barrier instead of a parity of o_done
     if (ok && total > 0 &&
-        !__all_sync(0xffffffffu,
-                    mbar_wait(smem_u32(&sm.bar_o_final), 0, abort_flag, status_word, 9)))
+        !__all_sync(0xffffffffu, mbar_wait(b_final, 0, abort_flag, status_word, 9)))
       ok = false;
     tc_fence_after();
 

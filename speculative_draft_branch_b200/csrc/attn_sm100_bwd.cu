@@ -12,15 +12,19 @@
 // Two kernels, neither with atomics:
 //   dq_sm100_kernel    query-stationary (one CTA per 128-row query tile and q
 //                      head, the forward's work order): per key tile S and dP
-//                      into TMEM, dS by 256 threads (two per row), dS into
-//                      shared memory, dQ += dS K accumulated in TMEM.
+//                      into TMEM, dS by 256 threads (two per row) written back
+//                      to TMEM as bf16, dQ += dS K (A operand from TMEM)
+//                      accumulated in TMEM; K and V come through separate
+//                      rings so V is refilled as soon as dP is done.
 //   dkdv_sm100_kernel  key-stationary (one CTA per 128-row key tile and kv
 //                      head, the plan's backward work order): over every
 //                      64-row query chunk of every q head of the group that
 //                      visits the tile, S^T = K Q^T and dP^T = V dO^T into
-//                      (double-buffered) TMEM, P^T and dS^T into shared
-//                      memory, dV += P^T dO and dK += dS^T Q accumulated in
-//                      TMEM for the whole walk.
+//                      double-buffered TMEM, P^T and dS^T written over them as
+//                      bf16, dV += P^T dO and dK += dS^T Q (A operands from
+//                      TMEM) accumulated in TMEM for the whole walk.  Per-query
+//                      records {LSE, D, key interval} arrive by bulk copy with
+//                      the Q / dO tiles through a 4-deep ring.
 #include "attn_sm100_common.cuh"
 
 namespace ba {
@@ -31,18 +35,21 @@ using namespace sm100;
 // ============================================================================
 // dQ kernel
 // ============================================================================
+constexpr int kDqKStages = 3;  // K is read twice (S, then dQ): deeper ring
+constexpr int kDqVStages = 2;  // V is free as soon as dP is computed
+
 template <int D>
 struct DqSmem {
   bf16 q[128 * D];
   bf16 dout[128 * D];
-  bf16 k[2][128 * D];
-  bf16 v[2][128 * D];
-  bf16 ds[128 * 128];  // dS: two [128 rows][64 keys] halves
+  bf16 k[kDqKStages][128 * D];
+  bf16 v[kDqVStages][128 * D];
   uint64_t bar_qdo;
-  uint64_t bar_kv_full[2], bar_kv_empty[2];
+  uint64_t bar_k_full[kDqKStages], bar_k_empty[kDqKStages];
+  uint64_t bar_v_full[kDqVStages], bar_v_empty[kDqVStages];
   uint64_t bar_sdp_full, bar_sdp_empty;
-  uint64_t bar_ds_full, bar_ds_empty;
-  uint64_t bar_dq_done;
+  uint64_t bar_ds_full[2];  // one per dS buffer: the dS threads may run a tile ahead
+  uint64_t bar_dq_final;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -52,6 +59,8 @@ struct DqMaps {
   CUtensorMap do_m, do_b;
 };
 
+// TMEM columns: S [0, 128), dP [128, 256), dQ [256, 256 + D), dS (bf16 pairs)
+// double-buffered at 384 and 448.
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     dq_sm100_kernel(const AttnParams a, const __grid_constant__ DqMaps tm) {
@@ -77,19 +86,22 @@ __global__ void __launch_bounds__(384, 1)
 
   const uint32_t b_qdo = smem_u32(&sm.bar_qdo);
   const uint32_t b_sdp_full = smem_u32(&sm.bar_sdp_full), b_sdp_empty = smem_u32(&sm.bar_sdp_empty);
-  const uint32_t b_ds_full = smem_u32(&sm.bar_ds_full), b_ds_empty = smem_u32(&sm.bar_ds_empty);
-  const uint32_t b_dq = smem_u32(&sm.bar_dq_done);
+  const uint32_t b_final = smem_u32(&sm.bar_dq_final);
   if (threadIdx.x == 0) {
     mbar_init(b_qdo, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&sm.bar_kv_full[s]), 1);
-      mbar_init(smem_u32(&sm.bar_kv_empty[s]), 1);
+    for (int s = 0; s < kDqKStages; ++s) {
+      mbar_init(smem_u32(&sm.bar_k_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_k_empty[s]), 1);
+    }
+    for (int s = 0; s < kDqVStages; ++s) {
+      mbar_init(smem_u32(&sm.bar_v_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_v_empty[s]), 1);
     }
     mbar_init(b_sdp_full, 1);
     mbar_init(b_sdp_empty, 256);
-    mbar_init(b_ds_full, 256);
-    mbar_init(b_ds_empty, 1);
-    mbar_init(b_dq, 1);
+    mbar_init(smem_u32(&sm.bar_ds_full[0]), 256);
+    mbar_init(smem_u32(&sm.bar_ds_full[1]), 256);
+    mbar_init(b_final, 1);
     sm.abort_flag = 0;
     mbar_fence_init();
   }
@@ -102,6 +114,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
+  auto t_ds = [&](int b) { return tmem + 384 + b * 64; };
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -115,59 +128,71 @@ __global__ void __launch_bounds__(384, 1)
         tma_load_3d(smem_u32(sm.dout) + x * 16384, dm, b_qdo, x * 64, h, row0);
       }
     }
-    int issued = 0;
+    int issued_k = 0, issued_v = 0;
     for (int j = 0; j < total; ++j) {
-      const int st = j & 1;
-      if (j >= 2 && !mbar_wait(smem_u32(&sm.bar_kv_empty[st]), ((j - 2) >> 1) & 1, abort_flag,
-                               status_word, 1))
-        break;
       int key0, kind;
       bool full;
       segs.locate(j, key0, kind, full);
-      const CUtensorMap *km = kind == 2 ? &tm.t.k_b : &tm.t.k_m;
-      const CUtensorMap *vm = kind == 2 ? &tm.t.v_b : &tm.t.v_m;
-      const uint32_t bar = smem_u32(&sm.bar_kv_full[st]);
-      mbar_expect_tx(bar, 2 * 128 * D * 2);
+      const int ks = j % kDqKStages, vs = j % kDqVStages;
+      if (j >= kDqKStages && !mbar_wait(smem_u32(&sm.bar_k_empty[ks]),
+                                        ((j / kDqKStages) - 1) & 1, abort_flag, status_word, 1))
+        break;
+      const uint32_t kb = smem_u32(&sm.bar_k_full[ks]);
+      mbar_expect_tx(kb, 128 * D * 2);
 #pragma unroll
-      for (int x = 0; x < D / 64; ++x) {
-        tma_load_3d(smem_u32(sm.k[st]) + x * 16384, km, bar, x * 64, g, key0);
-        tma_load_3d(smem_u32(sm.v[st]) + x * 16384, vm, bar, x * 64, g, key0);
-      }
-      ++issued;
+      for (int x = 0; x < D / 64; ++x)
+        tma_load_3d(smem_u32(sm.k[ks]) + x * 16384, kind == 2 ? &tm.t.k_b : &tm.t.k_m, kb, x * 64,
+                    g, key0);
+      ++issued_k;
+      if (j >= kDqVStages && !mbar_wait(smem_u32(&sm.bar_v_empty[vs]),
+                                        ((j / kDqVStages) - 1) & 1, abort_flag, status_word, 1))
+        break;
+      const uint32_t vb = smem_u32(&sm.bar_v_full[vs]);
+      mbar_expect_tx(vb, 128 * D * 2);
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x)
+        tma_load_3d(smem_u32(sm.v[vs]) + x * 16384, kind == 2 ? &tm.t.v_b : &tm.t.v_m, vb, x * 64,
+                    g, key0);
+      ++issued_v;
     }
-    for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-      mbar_wait(smem_u32(&sm.bar_kv_full[j & 1]), (j >> 1) & 1, abort_flag, status_word, 2);
+    for (int j = (issued_k > kDqKStages ? issued_k - kDqKStages : 0); j < issued_k; ++j)
+      mbar_wait(smem_u32(&sm.bar_k_full[j % kDqKStages]), (j / kDqKStages) & 1, abort_flag,
+                status_word, 2);
+    for (int j = (issued_v > kDqVStages ? issued_v - kDqVStages : 0); j < issued_v; ++j)
+      mbar_wait(smem_u32(&sm.bar_v_full[j % kDqVStages]), (j / kDqVStages) & 1, abort_flag,
+                status_word, 2);
     if (total > 0) mbar_wait(b_qdo, 0, abort_flag, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
     constexpr uint32_t idesc_dq = idesc_bf16(128, D, false, true);
     bool ok = total == 0 || mbar_wait(b_qdo, 0, abort_flag, status_word, 3);
-    const uint32_t q_s = smem_u32(sm.q), do_s = smem_u32(sm.dout), ds_s = smem_u32(sm.ds);
+    const uint32_t q_s = smem_u32(sm.q), do_s = smem_u32(sm.dout);
     auto issue_dq = [&](int i) -> bool {
-      if (!mbar_wait(b_ds_full, i & 1, abort_flag, status_word, 4)) return false;
+      if (!mbar_wait(smem_u32(&sm.bar_ds_full[i & 1]), (i >> 1) & 1, abort_flag, status_word, 4))
+        return false;
       tc_fence_after();
-      const uint32_t k_s = smem_u32(sm.k[i & 1]);
+      const uint32_t k_s = smem_u32(sm.k[i % kDqKStages]);
+      // dQ += dS K: dS (bf16 pairs) from TMEM, K as an MN-major operand
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint64_t ad = sdesc(ds_s + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-        const uint64_t bd = sdesc(k_s + k * 2048, 16384, 1024);
-        mma_bf16(t_dq, ad, bd, idesc_dq, (i > 0 || k > 0) ? 1u : 0u);
-      }
-      mma_commit(b_ds_empty);
-      mma_commit(smem_u32(&sm.bar_kv_empty[i & 1]));
-      mma_commit(b_dq);
+      for (int k = 0; k < 8; ++k)
+        mma_bf16_ts(t_dq, t_ds(i & 1) + k * 8, sdesc(k_s + k * 2048, 16384, 1024), idesc_dq,
+                    (i > 0 || k > 0) ? 1u : 0u);
+      mma_commit(smem_u32(&sm.bar_k_empty[i % kDqKStages]));
       return true;
     };
     for (int j = 0; ok && j < total; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(smem_u32(&sm.bar_kv_full[st]), (j >> 1) & 1, abort_flag, status_word, 5) ||
+      const int ks = j % kDqKStages, vs = j % kDqVStages;
+      if (!mbar_wait(smem_u32(&sm.bar_k_full[ks]), (j / kDqKStages) & 1, abort_flag, status_word,
+                     5) ||
+          !mbar_wait(smem_u32(&sm.bar_v_full[vs]), (j / kDqVStages) & 1, abort_flag, status_word,
+                     5) ||
           (j >= 1 && !mbar_wait(b_sdp_empty, (j - 1) & 1, abort_flag, status_word, 6))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t k_s = smem_u32(sm.k[st]), v_s = smem_u32(sm.v[st]);
+      const uint32_t k_s = smem_u32(sm.k[ks]), v_s = smem_u32(sm.v[vs]);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
@@ -181,12 +206,13 @@ __global__ void __launch_bounds__(384, 1)
                  k > 0 ? 1u : 0u);
       }
       mma_commit(b_sdp_full);
+      mma_commit(smem_u32(&sm.bar_v_empty[vs]));
       if (j >= 1 && !issue_dq(j - 1)) {
         ok = false;
         break;
       }
     }
-    if (ok && total > 0) issue_dq(total - 1);
+    if (ok && total > 0 && issue_dq(total - 1)) mma_commit(b_final);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ dS (2 threads / row)
     const int ew = threadIdx.x - 128;
@@ -203,8 +229,6 @@ __global__ void __launch_bounds__(384, 1)
       dd = a.d_all[(int64_t)h * ((int64_t)a.n_main + a.n_bt) + row_off + row0 + row];
     }
     bool ok = true;
-    const uint32_t swz = (uint32_t)(row & 7);
-    const uint32_t ds_row = smem_u32(sm.ds) + half * 16384 + row * 128;
     for (int j = 0; j < total; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(b_sdp_full, j & 1, abort_flag, status_word, 7))) {
         ok = false;
@@ -224,29 +248,28 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(b_sdp_empty);
       const int kbase = key0 + half * 64;
+      // dS packed to bf16 pairs in place (entry c/2 after entries c, c+1)
+      uint32_t *pk = reinterpret_cast<uint32_t *>(dp);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int key = kbase + c;
-        const bool vis = valid && (full || (key >= clo && key <= chi));
-        const float p = vis ? ex2(s[c] * a.scale_log2 - lse2) : 0.f;
-        dp[c] = p * (dp[c] - dd);
-      }
-      if (j >= 1 &&
-          !__all_sync(0xffffffffu, mbar_wait(b_ds_empty, (j - 1) & 1, abort_flag, status_word, 8))) {
-        ok = false;
-        break;
-      }
+      for (int c = 0; c < 64; c += 2) {
+        float d2[2];
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        st_shared_v4(ds_row + ((ch ^ swz) << 4), pack_bf16(dp[8 * ch], dp[8 * ch + 1]),
-                     pack_bf16(dp[8 * ch + 2], dp[8 * ch + 3]),
-                     pack_bf16(dp[8 * ch + 4], dp[8 * ch + 5]),
-                     pack_bf16(dp[8 * ch + 6], dp[8 * ch + 7]));
-      fence_proxy_async_smem();
-      mbar_arrive(b_ds_full);
+        for (int e = 0; e < 2; ++e) {
+          const int key = kbase + c + e;
+          const bool vis = valid && (full || (key >= clo && key <= chi));
+          const float p = vis ? ex2(s[c + e] * a.scale_log2 - lse2) : 0.f;
+          d2[e] = p * (dp[c + e] - dd);
+        }
+        pk[c / 2] = pack_bf16(d2[0], d2[1]);
+      }
+      // dS buffer j&1 was last read by dQ_{j-2}, which completed before S_j
+      tmem_st32(t_ds(j & 1) + lane_addr + half * 32, pk);
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.bar_ds_full[j & 1]));
     }
     if (ok && total > 0 &&
-        !__all_sync(0xffffffffu, mbar_wait(b_dq, (total - 1) & 1, abort_flag, status_word, 9)))
+        !__all_sync(0xffffffffu, mbar_wait(b_final, 0, abort_flag, status_word, 9)))
       ok = false;
     tc_fence_after();
     bf16 *dst = (is_main ? a.dq_out_m : a.dq_out_b) + ((int64_t)(row0 + row) * a.hq + h) * D +
@@ -285,23 +308,19 @@ __global__ void __launch_bounds__(384, 1)
 // ============================================================================
 // dK / dV kernel
 // ============================================================================
-constexpr int kQc = 64;  // query rows per chunk
+constexpr int kQc = 64;      // query rows per chunk
+constexpr int kKvStages = 4;  // Q / dO / record ring depth
 
 template <int D>
 struct DkvSmem {
   bf16 k[128 * D];
   bf16 v[128 * D];
-  bf16 q[2][kQc * D];        // D/64 boxes of [64 rows][64], 8 KB each
-  bf16 dout[2][kQc * D];
-  bf16 pt[2][128 * kQc];     // P^T  [128 keys][64 queries]
-  bf16 dst[2][128 * kQc];    // dS^T [128 keys][64 queries]
-  float lse2[2][kQc];        // LSE of each query, log2 units
-  float dd[2][kQc];          // D of each query
-  int lo[2][kQc], hi[2][kQc];  // key interval of each query (empty: lo > hi)
+  bf16 q[kKvStages][kQc * D];     // D/64 boxes of [64 rows][64], 8 KB each
+  bf16 dout[kKvStages][kQc * D];
+  float4 rec[kKvStages][kQc];     // {LSE log2, D, key lo, key hi} per query
   uint64_t bar_kv;
-  uint64_t bar_qdo_full[2], bar_qdo_empty[2], bar_vec_full[2];
-  uint64_t bar_sdp_full[2], bar_sdp_empty[2];
-  uint64_t bar_pds_full[2], bar_pds_empty[2];
+  uint64_t bar_qdo_full[kKvStages], bar_qdo_empty[kKvStages];
+  uint64_t bar_sdp_full[2], bar_pds_full[2];
   uint64_t bar_acc_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -327,6 +346,9 @@ struct ChunkWalk {
   }
 };
 
+// TMEM columns: dK [0, 128), dV [128, 256), S^T / P^T buffers at 256 and 320,
+// dP^T / dS^T buffers at 384 and 448 (P^T and dS^T, bf16, overwrite the first
+// 32 columns of the S^T / dP^T they are computed from).
 template <int D>
 __global__ void __launch_bounds__(256, 1)
     dkdv_sm100_kernel(const AttnParams a, const __grid_constant__ DkvMaps tm) {
@@ -356,19 +378,17 @@ __global__ void __launch_bounds__(256, 1)
   const int total = cw.grp * cw.per_head;
   int *status_word = a.plan.status + 1;
   volatile int *abort_flag = &sm.abort_flag;
-  const int64_t all_rows = (int64_t)a.n_main + a.n_bt;
 
   const uint32_t b_kv = smem_u32(&sm.bar_kv), b_acc = smem_u32(&sm.bar_acc_done);
   if (threadIdx.x == 0) {
     mbar_init(b_kv, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKvStages; ++s) {
       mbar_init(smem_u32(&sm.bar_qdo_full[s]), 1);
       mbar_init(smem_u32(&sm.bar_qdo_empty[s]), 1);
-      mbar_init(smem_u32(&sm.bar_vec_full[s]), 32);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&sm.bar_sdp_full[s]), 1);
-      mbar_init(smem_u32(&sm.bar_sdp_empty[s]), 128);
       mbar_init(smem_u32(&sm.bar_pds_full[s]), 128);
-      mbar_init(smem_u32(&sm.bar_pds_empty[s]), 1);
     }
     mbar_init(b_acc, 1);
     sm.abort_flag = 0;
@@ -385,11 +405,12 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t t_dk = tmem, t_dv = tmem + 128;
   auto t_s = [&](int b) { return tmem + 256 + b * 64; };
   auto t_dp = [&](int b) { return tmem + 384 + b * 64; };
+  // records of this CTA's key kind: main-key intervals or branch-local ones
+  const float4 *rec_base = a.rec + (main_kv ? 0 : (int64_t)a.hq * a.rows_pad);
 
-  if (warp == 0) {
+  if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    // lane 0 issues the TMA tile loads, all lanes stage the per-query vectors
-    if (lane == 0 && total > 0) {
+    if (total > 0) {
       mbar_expect_tx(b_kv, 2 * 128 * D * 2);
       const CUtensorMap *km = main_kv ? &tm.t.k_m : &tm.t.k_b;
       const CUtensorMap *vm = main_kv ? &tm.t.v_m : &tm.t.v_b;
@@ -401,53 +422,31 @@ __global__ void __launch_bounds__(256, 1)
     }
     int issued = 0;
     for (int c = 0; c < total; ++c) {
-      const int st = c & 1;
-      if (c >= 2 && !__all_sync(0xffffffffu,
-                                mbar_wait(smem_u32(&sm.bar_qdo_empty[st]), ((c - 2) >> 1) & 1,
-                                          abort_flag, status_word, 1)))
+      const int st = c % kKvStages;
+      if (c >= kKvStages &&
+          !mbar_wait(smem_u32(&sm.bar_qdo_empty[st]), ((c / kKvStages) - 1) & 1, abort_flag,
+                     status_word, 1))
         break;
       int h, tile, row0, nrows;
       bool is_main_q;
       cw.at(c, a, h, is_main_q, tile, row0, nrows);
-      if (lane == 0) {
-        const uint32_t bar = smem_u32(&sm.bar_qdo_full[st]);
-        mbar_expect_tx(bar, 2 * kQc * D * 2);
-        const CUtensorMap *qm = is_main_q ? &tm.q64_m : &tm.q64_b;
-        const CUtensorMap *dm = is_main_q ? &tm.do64_m : &tm.do64_b;
+      const uint32_t bar = smem_u32(&sm.bar_qdo_full[st]);
+      mbar_expect_tx(bar, 2 * kQc * D * 2 + kQc * 16);
+      const CUtensorMap *qm = is_main_q ? &tm.q64_m : &tm.q64_b;
+      const CUtensorMap *dm = is_main_q ? &tm.do64_m : &tm.do64_b;
 #pragma unroll
-        for (int x = 0; x < D / 64; ++x) {
-          tma_load_3d(smem_u32(sm.q[st]) + x * 8192, qm, bar, x * 64, h, row0);
-          tma_load_3d(smem_u32(sm.dout[st]) + x * 8192, dm, bar, x * 64, h, row0);
-        }
+      for (int x = 0; x < D / 64; ++x) {
+        tma_load_3d(smem_u32(sm.q[st]) + x * 8192, qm, bar, x * 64, h, row0);
+        tma_load_3d(smem_u32(sm.dout[st]) + x * 8192, dm, bar, x * 64, h, row0);
       }
-      const int rows = is_main_q ? a.n_main : a.n_bt;
-      const int roff = is_main_q ? 0 : a.n_main;
-      const float *lse = is_main_q ? a.lse_m : a.lse_b;
-#pragma unroll
-      for (int i = 0; i < kQc / 32; ++i) {
-        const int r = lane + 32 * i;
-        float l2 = 0.f, dv = 0.f;
-        int lo = 1, hi = 0;
-        if (r < nrows) {
-          l2 = lse[(int64_t)h * rows + row0 + r] * kLog2e;
-          dv = a.d_all[(int64_t)h * all_rows + roff + row0 + r];
-          const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[roff + row0 + r];
-          lo = main_kv ? iv.x : iv.z;
-          hi = main_kv ? iv.y : iv.w;
-        }
-        sm.lse2[st][r] = l2;
-        sm.dd[st][r] = dv;
-        sm.lo[st][r] = lo;
-        sm.hi[st][r] = hi;
-      }
-      mbar_arrive(smem_u32(&sm.bar_vec_full[st]));
+      const int64_t prow = (is_main_q ? 0 : a.n_main_pad) + row0;
+      bulk_load(smem_u32(sm.rec[st]), rec_base + (int64_t)h * a.rows_pad + prow, kQc * 16, bar);
       ++issued;
     }
-    if (lane == 0) {
-      for (int c = (issued > 2 ? issued - 2 : 0); c < issued; ++c)
-        mbar_wait(smem_u32(&sm.bar_qdo_full[c & 1]), (c >> 1) & 1, abort_flag, status_word, 2);
-      if (total > 0) mbar_wait(b_kv, 0, abort_flag, status_word, 2);
-    }
+    for (int c = (issued > kKvStages ? issued - kKvStages : 0); c < issued; ++c)
+      mbar_wait(smem_u32(&sm.bar_qdo_full[c % kKvStages]), (c / kKvStages) & 1, abort_flag,
+                status_word, 2);
+    if (total > 0) mbar_wait(b_kv, 0, abort_flag, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_s = idesc_bf16(128, kQc, false, false);
@@ -455,49 +454,49 @@ __global__ void __launch_bounds__(256, 1)
     bool ok = total == 0 || mbar_wait(b_kv, 0, abort_flag, status_word, 3);
     const uint32_t k_s = smem_u32(sm.k), v_s = smem_u32(sm.v);
     auto grads = [&](int i) -> bool {
-      const int sb = i & 1;
+      const int sb = i & 1, st = i % kKvStages;
       if (!mbar_wait(smem_u32(&sm.bar_pds_full[sb]), (i >> 1) & 1, abort_flag, status_word, 4))
         return false;
       tc_fence_after();
-      const uint32_t p_s = smem_u32(sm.pt[sb]), ds_s = smem_u32(sm.dst[sb]);
-      const uint32_t q_s = smem_u32(sm.q[sb]), do_s = smem_u32(sm.dout[sb]);
+      const uint32_t q_s = smem_u32(sm.q[st]), do_s = smem_u32(sm.dout[st]);
+      // dV += P^T dO, dK += dS^T Q (P^T, dS^T from TMEM; K = 64 queries)
 #pragma unroll
       for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16(t_dv, sdesc(p_s + k * 32, 16, 1024), sdesc(do_s + k * 2048, 8192, 1024), idesc_g,
-                 (i > 0 || k > 0) ? 1u : 0u);
+        mma_bf16_ts(t_dv, t_s(sb) + k * 8, sdesc(do_s + k * 2048, 8192, 1024), idesc_g,
+                    (i > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
       for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16(t_dk, sdesc(ds_s + k * 32, 16, 1024), sdesc(q_s + k * 2048, 8192, 1024), idesc_g,
-                 (i > 0 || k > 0) ? 1u : 0u);
-      mma_commit(smem_u32(&sm.bar_pds_empty[sb]));
-      mma_commit(smem_u32(&sm.bar_qdo_empty[sb]));
+        mma_bf16_ts(t_dk, t_dp(sb) + k * 8, sdesc(q_s + k * 2048, 8192, 1024), idesc_g,
+                    (i > 0 || k > 0) ? 1u : 0u);
+      mma_commit(smem_u32(&sm.bar_qdo_empty[st]));
       return true;
     };
     for (int c = 0; ok && c < total; ++c) {
-      const int st = c & 1;
-      if (!mbar_wait(smem_u32(&sm.bar_qdo_full[st]), (c >> 1) & 1, abort_flag, status_word, 5) ||
-          (c >= 2 && !mbar_wait(smem_u32(&sm.bar_sdp_empty[st]), ((c - 2) >> 1) & 1, abort_flag,
-                                status_word, 6))) {
+      const int st = c % kKvStages, sb = c & 1;
+      if (!mbar_wait(smem_u32(&sm.bar_qdo_full[st]), (c / kKvStages) & 1, abort_flag, status_word,
+                     5)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      // S^T / dP^T buffer sb was last read (as P^T / dS^T) by grads(c - 2),
+      // issued before this point: tcgen05 MMAs of one thread run in order
       const uint32_t q_s = smem_u32(sm.q[st]), do_s = smem_u32(sm.dout[st]);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
         const uint32_t qa = (k >> 2) * 8192 + (k & 3) * 32;
-        mma_bf16(t_s(st), sdesc(k_s + ka, 16, 1024), sdesc(q_s + qa, 16, 1024), idesc_s,
+        mma_bf16(t_s(sb), sdesc(k_s + ka, 16, 1024), sdesc(q_s + qa, 16, 1024), idesc_s,
                  k > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
         const uint32_t qa = (k >> 2) * 8192 + (k & 3) * 32;
-        mma_bf16(t_dp(st), sdesc(v_s + ka, 16, 1024), sdesc(do_s + qa, 16, 1024), idesc_s,
+        mma_bf16(t_dp(sb), sdesc(v_s + ka, 16, 1024), sdesc(do_s + qa, 16, 1024), idesc_s,
                  k > 0 ? 1u : 0u);
       }
-      mma_commit(smem_u32(&sm.bar_sdp_full[st]));
+      mma_commit(smem_u32(&sm.bar_sdp_full[sb]));
       if (c >= 1 && !grads(c - 1)) {
         ok = false;
         break;
@@ -509,56 +508,46 @@ __global__ void __launch_bounds__(256, 1)
     const int row = threadIdx.x - 128;
     const int key = key0 + row;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t swz = (uint32_t)(row & 7);
     bool ok = true;
     for (int c = 0; c < total; ++c) {
-      const int st = c & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_sdp_full[st]), (c >> 1) & 1,
-                                             abort_flag, status_word, 7))) {
+      const int st = c % kKvStages, sb = c & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_sdp_full[sb]), (c >> 1) & 1,
+                                             abort_flag, status_word, 7)) ||
+          !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_qdo_full[st]),
+                                             (c / kKvStages) & 1, abort_flag, status_word, 8))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[kQc], dp[kQc];
-      tmem_ld32(t_s(st) + lane_addr, reinterpret_cast<uint32_t *>(s));
-      tmem_ld32(t_s(st) + lane_addr + 32, reinterpret_cast<uint32_t *>(s) + 32);
-      tmem_ld32(t_dp(st) + lane_addr, reinterpret_cast<uint32_t *>(dp));
-      tmem_ld32(t_dp(st) + lane_addr + 32, reinterpret_cast<uint32_t *>(dp) + 32);
-      tc_wait_ld();
+      // two passes of 32 queries: P^T / dS^T (bf16 pairs) overwrite the
+      // first 32 columns of S^T / dP^T, which the first pass has consumed
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        float s[32], dp[32];
+        tmem_ld32(t_s(sb) + lane_addr + pass * 32, reinterpret_cast<uint32_t *>(s));
+        tmem_ld32(t_dp(sb) + lane_addr + pass * 32, reinterpret_cast<uint32_t *>(dp));
+        tc_wait_ld();
+        uint32_t pk[16], dk2[16];
+#pragma unroll
+        for (int q = 0; q < 32; q += 2) {
+          float p2[2], d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float4 r = sm.rec[st][pass * 32 + q + e];
+            const bool vis = key >= __float_as_int(r.z) && key <= __float_as_int(r.w);
+            const float p = vis ? ex2(s[q + e] * a.scale_log2 - r.x) : 0.f;
+            p2[e] = p;
+            d2[e] = p * (dp[q + e] - r.y);
+          }
+          pk[q / 2] = pack_bf16(p2[0], p2[1]);
+          dk2[q / 2] = pack_bf16(d2[0], d2[1]);
+        }
+        tmem_st16(t_s(sb) + lane_addr + pass * 16, pk);
+        tmem_st16(t_dp(sb) + lane_addr + pass * 16, dk2);
+      }
+      tc_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.bar_sdp_empty[st]));
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_vec_full[st]), (c >> 1) & 1,
-                                             abort_flag, status_word, 8))) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int q = 0; q < kQc; ++q) {
-        const bool vis = key >= sm.lo[st][q] && key <= sm.hi[st][q];
-        const float p = vis ? ex2(s[q] * a.scale_log2 - sm.lse2[st][q]) : 0.f;
-        s[q] = p;
-        dp[q] = p * (dp[q] - sm.dd[st][q]);
-      }
-      if (c >= 2 && !__all_sync(0xffffffffu,
-                                mbar_wait(smem_u32(&sm.bar_pds_empty[st]), ((c - 2) >> 1) & 1,
-                                          abort_flag, status_word, 9))) {
-        ok = false;
-        break;
-      }
-      const uint32_t p_row = smem_u32(sm.pt[st]) + row * 128;
-      const uint32_t d_row = smem_u32(sm.dst[st]) + row * 128;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        st_shared_v4(p_row + ((ch ^ swz) << 4), pack_bf16(s[8 * ch], s[8 * ch + 1]),
-                     pack_bf16(s[8 * ch + 2], s[8 * ch + 3]), pack_bf16(s[8 * ch + 4], s[8 * ch + 5]),
-                     pack_bf16(s[8 * ch + 6], s[8 * ch + 7]));
-        st_shared_v4(d_row + ((ch ^ swz) << 4), pack_bf16(dp[8 * ch], dp[8 * ch + 1]),
-                     pack_bf16(dp[8 * ch + 2], dp[8 * ch + 3]),
-                     pack_bf16(dp[8 * ch + 4], dp[8 * ch + 5]),
-                     pack_bf16(dp[8 * ch + 6], dp[8 * ch + 7]));
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(&sm.bar_pds_full[st]));
+      mbar_arrive(smem_u32(&sm.bar_pds_full[sb]));
     }
     if (ok && total > 0 &&
         !__all_sync(0xffffffffu, mbar_wait(b_acc, 0, abort_flag, status_word, 10)))

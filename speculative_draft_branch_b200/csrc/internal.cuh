@@ -41,6 +41,11 @@ struct AttnParams {
   __nv_bfloat16 *dk_m, *dv_m, *dk_b, *dv_b;
   __nv_bfloat16 *dq_out_m, *dq_out_b;  // dQ written directly (tcgen05 backward)
   int32_t zero_dq_acc;                  // preprocess clears dq_acc (mma.sync backward)
+  // per-query backward records {LSE * log2(e), D, key lo, key hi} (tcgen05
+  // backward): rec[kind][h][padded row], kind 0 = main-key interval, 1 =
+  // branch-local interval; main rows at [0, n_main_pad), branch rows after.
+  float4 *rec;
+  int32_t n_main_pad, rows_pad;
   // zigzag partial output (fp32 O accumulator [(N+Nb), Hq, d], LSE [Hq, N+Nb])
   float *zz_o;
   float *zz_lse;

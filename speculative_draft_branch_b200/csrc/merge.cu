@@ -135,7 +135,35 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(AttnParams a) {
     }
 #pragma unroll
     for (int o2 = kLanes / 2; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
-    if (active && lane == 0) const_cast<float *>(a.d_all)[(int64_t)h * rows + row] = s;
+    if (active && lane == 0) {
+      const_cast<float *>(a.d_all)[(int64_t)h * rows + row] = s;
+      if (a.rec) {
+        const bool is_main = row < a.n_main;
+        const int64_t r = is_main ? row : row - a.n_main;
+        const float l2 = (is_main ? a.lse_m : a.lse_b)[(int64_t)h * (is_main ? a.n_main : a.n_bt) + r] *
+                         1.4426950408889634f;
+        const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[row];
+        const int64_t pr = (is_main ? 0 : a.n_main_pad) + r;
+        a.rec[(int64_t)h * a.rows_pad + pr] =
+            make_float4(l2, s, __int_as_float(iv.x), __int_as_float(iv.y));
+        a.rec[((int64_t)a.hq + h) * a.rows_pad + pr] =
+            make_float4(l2, s, __int_as_float(iv.z), __int_as_float(iv.w));
+      }
+    }
+  }
+  // padding rows of the records: empty key intervals
+  if (a.rec) {
+    const int pad_m = a.n_main_pad - a.n_main;
+    const int pad_b = a.rows_pad - a.n_main_pad - a.n_bt;
+    const int64_t n_pad = (int64_t)(pad_m + pad_b) * a.hq * 2;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_pad;
+         i += (int64_t)gridDim.x * blockDim.x) {
+      const int per = pad_m + pad_b;
+      const int64_t kh = i / per;
+      const int j = (int)(i % per);
+      const int64_t pr = j < pad_m ? a.n_main + j : a.n_main_pad + a.n_bt + (j - pad_m);
+      a.rec[kh * a.rows_pad + pr] = make_float4(0.f, 0.f, __int_as_float(1), __int_as_float(0));
+    }
   }
 }
 

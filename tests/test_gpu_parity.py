@@ -65,6 +65,8 @@ def run(ba, st, t, family=0, bwd=True, zigzag_C=None):
         out = runner.forward(t)
         grads = runner.backward(t, out) if bwd else None
         torch.cuda.synchronize()
+        # raises BranchAttnError(BA_ERR_DEVICE_TIMEOUT) if a bounded wait gave up
+        assert runner.plan_status() == 0
     finally:
         ba.ba_set_kernel_family(0)
     return runner, out, grads
