@@ -233,6 +233,15 @@ BA_API ba_status lse_merge(int64_t rows, int32_t heads, int32_t head_dim,
                     const void *o_b, const float *lse_b, void *o_out,
                     float *lse_out, ba_stream_t stream);
 
+/* Device self-check of the exponential used by the softmax (no counterpart
+ * in the paper).  The forward softmax evaluates part of its 2^x on the FMA
+ * pipe with a range-reduced cubic (max relative error 7.5e-5) and the rest on
+ * the hardware ex2 unit; this call writes both for n inputs x (device
+ * pointers, fp32): y_fma[i] = polynomial 2^x[i], y_hw[i] = ex2.approx(x[i]).
+ * Inputs below -125 (and -inf) give y_fma = 0. */
+BA_API ba_status ba_exp2_check(const float *x, float *y_fma, float *y_hw, int64_t n,
+                               ba_stream_t stream);
+
 /* Kernel family for the attention kernels:
  *   0 = default (tcgen05/TMEM/TMA kernels),
  *   1 = tcgen05/TMEM/TMA kernels,

@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "BA_OK", -1: "BA_ERR_INVALID_ARG", -2: "BA_ERR_UNSUPPORTED",
 EXPORTS = ("ba_workspace_size", "ba_plan_layout_query", "ba_plan", "ba_plan_status",
            "branch_attn_fwd", "branch_attn_bwd", "lse_merge", "ba_set_kernel_family",
            "ba_get_kernel_family", "ba_set_kernel_events", "ba_launch_count", "ba_last_error",
-           "ba_version", "branch_attn_bwd_static_scratch")
+           "ba_version", "branch_attn_bwd_static_scratch", "ba_exp2_check")
 
 
 class BAProblem(ctypes.Structure):
@@ -78,6 +78,7 @@ def _load() -> ctypes.CDLL:
         "ba_set_kernel_family": [I32],
         "ba_get_kernel_family": [],
         "ba_set_kernel_events": [I32, VP, VP],
+        "ba_exp2_check": [VP, VP, VP, I64, VP],
         "ba_launch_count": [],
         "ba_last_error": [],
         "ba_version": [],
@@ -289,6 +290,15 @@ def ba_set_kernel_events(which: int, start=None, stop=None) -> None:
     """Record torch.cuda.Event `start`/`stop` around the fwd (0) / bwd (1) kernel."""
     _check(lib.ba_set_kernel_events(which, start.cuda_event if start is not None else None,
                                     stop.cuda_event if stop is not None else None))
+
+
+def ba_exp2_check(x, stream=None):
+    """(polynomial 2^x, hardware ex2) of a CUDA fp32 tensor, computed on the device."""
+    import torch
+    _expect(x, (x.numel(),), torch.float32, "x")
+    y_fma, y_hw = torch.empty_like(x), torch.empty_like(x)
+    _check(lib.ba_exp2_check(_ptr(x), _ptr(y_fma), _ptr(y_hw), x.numel(), _stream(stream)))
+    return y_fma, y_hw
 
 
 def ba_launch_count() -> int:

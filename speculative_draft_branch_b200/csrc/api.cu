@@ -418,6 +418,18 @@ ba_status lse_merge(int64_t rows, int32_t heads, int32_t head_dim, int32_t o_is_
                           o_out, lse_out, (cudaStream_t)stream);
 }
 
+ba_status ba_exp2_check(const float *x, float *y_fma, float *y_hw, int64_t n, ba_stream_t stream) {
+  if (n < 0) {
+    set_error("ba_exp2_check: n must be >= 0");
+    return BA_ERR_INVALID_ARG;
+  }
+  if (n == 0) return BA_OK;
+  BA_TRY(check_f32(x, true, "x"));
+  BA_TRY(check_f32(y_fma, true, "y_fma"));
+  BA_TRY(check_f32(y_hw, true, "y_hw"));
+  return launch_exp2_check(x, y_fma, y_hw, n, (cudaStream_t)stream);
+}
+
 ba_status ba_set_kernel_family(int32_t family) {
   if (family < 0 || family > 2) {
     set_error("unknown kernel family %d", family);

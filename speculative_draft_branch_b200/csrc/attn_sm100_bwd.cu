@@ -248,16 +248,23 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(b_sdp_empty);
       const int kbase = key0 + half * 64;
-      // dS packed to bf16 pairs in place (entry c/2 after entries c, c+1)
+      // masked scores -> -inf only on partial tiles, then P = 2^(s sl2 - l2)
+      // branch-free; dS packed to bf16 pairs in place (entry c/2 after c, c+1)
+      if (!(full && valid)) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int key = kbase + c;
+          if (key < clo || key > chi) s[c] = kNegInf;
+        }
+      }
+      const float sl2 = a.scale_log2;
       uint32_t *pk = reinterpret_cast<uint32_t *>(dp);
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
         float d2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int key = kbase + c + e;
-          const bool vis = valid && (full || (key >= clo && key <= chi));
-          const float p = vis ? ex2(s[c + e] * a.scale_log2 - lse2) : 0.f;
+          const float p = ex2(fmaf(s[c + e], sl2, -lse2));
           d2[e] = p * (dp[c + e] - dd);
         }
         pk[c / 2] = pack_bf16(d2[0], d2[1]);
@@ -508,9 +515,20 @@ __global__ void __launch_bounds__(256, 1)
     const int row = threadIdx.x - 128;
     const int key = key0 + row;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    const float sl2 = a.scale_log2;
     bool ok = true;
     for (int c = 0; c < total; ++c) {
       const int st = c % kKvStages, sb = c & 1;
+      // a chunk whose every query sees every key of this tile needs no mask
+      bool full = false;
+      if (main_kv) {
+        int h, tile, row0, nrows;
+        bool is_main_q;
+        cw.at(c, a, h, is_main_q, tile, row0, nrows);
+        const int32_t *qt =
+            a.plan.qtile + (int64_t)(is_main_q ? tile : a.n_qt_main + tile) * 6;
+        full = nrows == kQc && kt >= qt[1] && kt < qt[2];
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_sdp_full[sb]), (c >> 1) & 1,
                                              abort_flag, status_word, 7)) ||
           !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_qdo_full[st]),
@@ -528,14 +546,21 @@ __global__ void __launch_bounds__(256, 1)
         tmem_ld32(t_dp(sb) + lane_addr + pass * 32, reinterpret_cast<uint32_t *>(dp));
         tc_wait_ld();
         uint32_t pk[16], dk2[16];
+        if (!full) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const int2 iv = *reinterpret_cast<const int2 *>(
+                reinterpret_cast<const char *>(&sm.rec[st][pass * 32 + q]) + 8);
+            if (key < iv.x || key > iv.y) s[q] = kNegInf;
+          }
+        }
 #pragma unroll
         for (int q = 0; q < 32; q += 2) {
           float p2[2], d2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float4 r = sm.rec[st][pass * 32 + q + e];
-            const bool vis = key >= __float_as_int(r.z) && key <= __float_as_int(r.w);
-            const float p = vis ? ex2(s[q + e] * a.scale_log2 - r.x) : 0.f;
+            const float2 r = *reinterpret_cast<const float2 *>(&sm.rec[st][pass * 32 + q + e]);
+            const float p = ex2(fmaf(s[q + e], sl2, -r.x));
             p2[e] = p;
             d2[e] = p * (dp[q + e] - r.y);
           }

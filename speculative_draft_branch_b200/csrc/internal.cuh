@@ -86,6 +86,8 @@ bool sm100_fwd_available();
 bool sm100_bwd_available();
 ba_status launch_fwd_sm100(const AttnParams &a, cudaStream_t s);
 ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s);
+ba_status launch_exp2_check(const float *x, float *y_fma, float *y_mufu, int64_t n,
+                            cudaStream_t s);
 
 __host__ __device__ inline int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

@@ -216,10 +216,40 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
          ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Per-warpgroup register budget changes (all four warps of a warpgroup run
+// them, warp-uniformly).  The sum over warpgroups must fit the registers the
+// CTA was launched with.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x evaluated on the FMA / integer pipes, to take part of the exponentials
+// off the 16-per-clock MUFU unit.  Range reduction: n = round(x) by adding
+// 1.5 * 2^23 (the sum's low mantissa bits hold n), f = x - n in [-1/2, 1/2];
+// 2^f by a cubic fitted for minimax relative error (exp2_poly_fit.py: max
+// relative error 7.5e-5 in fp32); 2^n by adding n to the exponent field.
+// Inputs below -125 (including -inf) give 0.
+__device__ __forceinline__ float exp2_fma(float x) {
+  const float kShift = 12582912.0f;  // 1.5 * 2^23
+  const float t = x + kShift;
+  const float f = x - (t - kShift);
+  const float p = fmaf(fmaf(fmaf(0.055171623826026917f, f, 0.2426111251115799f), f,
+                            0.6932609677314758f),
+                       f, 0.9999280571937561f);
+  const int n = __float_as_int(t) - 0x4B400000;
+  const float r = __int_as_float(__float_as_int(p) + (n << 23));
+  return x < -125.0f ? 0.0f : r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

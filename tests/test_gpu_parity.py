@@ -332,3 +332,24 @@ def test_workload_ttt_256k_truncated_prefix(cuda_lib):
     km = oracle.keys_backward(st, t, main_keys=mkeys, groups=[0, 7])
     check("dk_m tail", cpu(g["dk_m"][mkeys][:, [0, 7]]), km["dk_m"][:, [0, 7]])
     check("dv_m tail", cpu(g["dv_m"][mkeys][:, [0, 7]]), km["dv_m"][:, [0, 7]])
+
+
+# ------------------------------------------------------------ exponential
+def test_exp2_polynomial_against_exact(cuda_lib):
+    """The FMA-pipe 2^x: relative error <= 1e-4 against exact 2^x (fp64) on the
+    softmax's input range, exactly 0 below -125, and the hardware ex2 within
+    about 2^-22 (checked at 1e-6) for reference."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001),
+                   torch.tensor([-125.0, -124.5, -0.5, -0.25, 0.0, 0.5, 1.0, 7.5, 8.0]),
+                   torch.tensor([-126.0, -200.0, -1e30, float("-inf")])]).float().cuda()
+    y_fma, y_hw = cuda_lib.ba_exp2_check(x)
+    xs = x.double().cpu().numpy()
+    exact = np.exp2(xs)
+    got = y_fma.double().cpu().numpy()
+    inside = xs >= -125.0
+    rel = np.abs(got[inside] / exact[inside] - 1.0)
+    assert rel.max() <= 1e-4, rel.max()
+    assert np.all(got[~inside] == 0.0)
+    hw = y_hw.double().cpu().numpy()
+    rel_hw = np.abs(hw[inside & (xs > -120)] / exact[inside & (xs > -120)] - 1.0)
+    assert rel_hw.max() <= 1e-6
