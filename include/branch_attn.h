@@ -206,9 +206,10 @@ BA_API ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws,
  * reserves its whole HBM budget in its own pool at start-up, or a plugin whose
  * host forbids allocation at run time) and cannot cudaMalloc the backward
  * workspace.  This call takes the same arguments as branch_attn_bwd minus the
- * workspace and keeps its scratch (D and the fp32 dQ accumulator) in a
- * 32 MiB array compiled into the library, which every GPU that loads the
- * library holds until exit.  It allocates nothing.
+ * workspace and keeps its scratch (D plus the fp32 dQ accumulator or the
+ * per-query backward records) in a 32 MiB array compiled into the library,
+ * which every GPU that loads the library holds until exit.  It allocates
+ * nothing.
  *   - Problems whose backward scratch (see ba_workspace_size) exceeds 32 MiB
  *     are rejected with BA_ERR_WORKSPACE_TOO_SMALL before any launch.
  *   - The first call on a device looks up the array's device address (with

@@ -354,10 +354,12 @@ struct ChunkWalk {
 };
 
 // TMEM columns: dK [0, 128), dV [128, 256), S^T / P^T buffers at 256 and 320,
-// dP^T / dS^T buffers at 384 and 448 (P^T and dS^T, bf16, overwrite the first
-// 32 columns of the S^T / dP^T they are computed from).
+// dP^T / dS^T buffers at 384 and 448.  Two threads per key row: the thread for
+// queries [32h, 32h + 32) writes their P^T / dS^T (bf16 pairs) over columns
+// [32h, 32h + 16) of the S^T / dP^T it read, so K-step k (16 queries) of the
+// dV / dK products sits at column (k / 2) * 32 + (k % 2) * 8.
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     dkdv_sm100_kernel(const AttnParams a, const __grid_constant__ DkvMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -395,7 +397,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&sm.bar_sdp_full[s]), 1);
-      mbar_init(smem_u32(&sm.bar_pds_full[s]), 128);
+      mbar_init(smem_u32(&sm.bar_pds_full[s]), 256);
     }
     mbar_init(b_acc, 1);
     sm.abort_flag = 0;
@@ -469,12 +471,12 @@ __global__ void __launch_bounds__(256, 1)
       // dV += P^T dO, dK += dS^T Q (P^T, dS^T from TMEM; K = 64 queries)
 #pragma unroll
       for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16_ts(t_dv, t_s(sb) + k * 8, sdesc(do_s + k * 2048, 8192, 1024), idesc_g,
-                    (i > 0 || k > 0) ? 1u : 0u);
+        mma_bf16_ts(t_dv, t_s(sb) + (k >> 1) * 32 + (k & 1) * 8,
+                    sdesc(do_s + k * 2048, 8192, 1024), idesc_g, (i > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
       for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16_ts(t_dk, t_dp(sb) + k * 8, sdesc(q_s + k * 2048, 8192, 1024), idesc_g,
-                    (i > 0 || k > 0) ? 1u : 0u);
+        mma_bf16_ts(t_dk, t_dp(sb) + (k >> 1) * 32 + (k & 1) * 8,
+                    sdesc(q_s + k * 2048, 8192, 1024), idesc_g, (i > 0 || k > 0) ? 1u : 0u);
       mma_commit(smem_u32(&sm.bar_qdo_empty[st]));
       return true;
     };
@@ -511,8 +513,10 @@ __global__ void __launch_bounds__(256, 1)
     }
     if (ok && total > 0 && grads(total - 1)) mma_commit(b_acc);
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ P^T, dS^T (1 thread / key)
-    const int row = threadIdx.x - 128;
+    // ------------------------------------------------------------ P^T, dS^T (2 threads / key)
+    const int ew = threadIdx.x - 128;
+    const int qh = ew >> 7;           // query half: [32 qh, 32 qh + 32)
+    const int row = ew & 127;
     const int key = key0 + row;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
@@ -537,39 +541,35 @@ __global__ void __launch_bounds__(256, 1)
         break;
       }
       tc_fence_after();
-      // two passes of 32 queries: P^T / dS^T (bf16 pairs) overwrite the
-      // first 32 columns of S^T / dP^T, which the first pass has consumed
+      float s[32], dp[32];
+      tmem_ld32(t_s(sb) + lane_addr + qh * 32, reinterpret_cast<uint32_t *>(s));
+      tmem_ld32(t_dp(sb) + lane_addr + qh * 32, reinterpret_cast<uint32_t *>(dp));
+      tc_wait_ld();
+      const float4 *rec = sm.rec[st] + qh * 32;
+      if (!full) {
 #pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        float s[32], dp[32];
-        tmem_ld32(t_s(sb) + lane_addr + pass * 32, reinterpret_cast<uint32_t *>(s));
-        tmem_ld32(t_dp(sb) + lane_addr + pass * 32, reinterpret_cast<uint32_t *>(dp));
-        tc_wait_ld();
-        uint32_t pk[16], dk2[16];
-        if (!full) {
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int2 iv = *reinterpret_cast<const int2 *>(
-                reinterpret_cast<const char *>(&sm.rec[st][pass * 32 + q]) + 8);
-            if (key < iv.x || key > iv.y) s[q] = kNegInf;
-          }
+        for (int q = 0; q < 32; ++q) {
+          const int2 iv =
+              *reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(&rec[q]) + 8);
+          if (key < iv.x || key > iv.y) s[q] = kNegInf;
         }
-#pragma unroll
-        for (int q = 0; q < 32; q += 2) {
-          float p2[2], d2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float2 r = *reinterpret_cast<const float2 *>(&sm.rec[st][pass * 32 + q + e]);
-            const float p = ex2(fmaf(s[q + e], sl2, -r.x));
-            p2[e] = p;
-            d2[e] = p * (dp[q + e] - r.y);
-          }
-          pk[q / 2] = pack_bf16(p2[0], p2[1]);
-          dk2[q / 2] = pack_bf16(d2[0], d2[1]);
-        }
-        tmem_st16(t_s(sb) + lane_addr + pass * 16, pk);
-        tmem_st16(t_dp(sb) + lane_addr + pass * 16, dk2);
       }
+      uint32_t pk[16], dk2[16];
+#pragma unroll
+      for (int q = 0; q < 32; q += 2) {
+        float p2[2], d2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float2 r = *reinterpret_cast<const float2 *>(&rec[q + e]);
+          const float p = ex2(fmaf(s[q + e], sl2, -r.x));
+          p2[e] = p;
+          d2[e] = p * (dp[q + e] - r.y);
+        }
+        pk[q / 2] = pack_bf16(p2[0], p2[1]);
+        dk2[q / 2] = pack_bf16(d2[0], d2[1]);
+      }
+      tmem_st16(t_s(sb) + lane_addr + qh * 32, pk);
+      tmem_st16(t_dp(sb) + lane_addr + qh * 32, dk2);
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.bar_pds_full[sb]));
@@ -578,16 +578,17 @@ __global__ void __launch_bounds__(256, 1)
         !__all_sync(0xffffffffu, mbar_wait(b_acc, 0, abort_flag, status_word, 10)))
       ok = false;
     tc_fence_after();
+    // epilogue: each of the two threads of a key row stores half of dK and dV
     const bool valid = key < n_keys;
-    bf16 *dkg = (main_kv ? a.dk_m : a.dk_b) + ((int64_t)key * a.hkv + g) * D;
-    bf16 *dvg = (main_kv ? a.dv_m : a.dv_b) + ((int64_t)key * a.hkv + g) * D;
+    bf16 *dkg = (main_kv ? a.dk_m : a.dk_b) + ((int64_t)key * a.hkv + g) * D + qh * (D / 2);
+    bf16 *dvg = (main_kv ? a.dv_m : a.dv_b) + ((int64_t)key * a.hkv + g) * D + qh * (D / 2);
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
-      const uint32_t src = part == 0 ? t_dk : t_dv;
+      const uint32_t src = (part == 0 ? t_dk : t_dv) + qh * (D / 2);
       const float mul = part == 0 ? a.scale : 1.f;
       bf16 *dst = part == 0 ? dkg : dvg;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
         if (ok && total > 0) {
           tmem_ld32(src + lane_addr + c * 32, o);
@@ -666,13 +667,13 @@ ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s) {
   const int64_t grid_dq = (int64_t)a.n_qt * a.hq;
   const int64_t grid_kv = (int64_t)(a.n_kt + a.n_bkt) * a.hkv;
   if (d == 64) {
-    if ((st = launch_kernel(dkdv_sm100_kernel<64>, sizeof(DkvSmem<64>) + 1024, grid_kv, 256, a,
+    if ((st = launch_kernel(dkdv_sm100_kernel<64>, sizeof(DkvSmem<64>) + 1024, grid_kv, 384, a,
                             kvm, s, "dkdv_sm100_kernel<64>")) != BA_OK)
       return st;
     return launch_kernel(dq_sm100_kernel<64>, sizeof(DqSmem<64>) + 1024, grid_dq, 384, a, dqm, s,
                          "dq_sm100_kernel<64>");
   }
-  if ((st = launch_kernel(dkdv_sm100_kernel<128>, sizeof(DkvSmem<128>) + 1024, grid_kv, 256, a,
+  if ((st = launch_kernel(dkdv_sm100_kernel<128>, sizeof(DkvSmem<128>) + 1024, grid_kv, 384, a,
                           kvm, s, "dkdv_sm100_kernel<128>")) != BA_OK)
     return st;
   return launch_kernel(dq_sm100_kernel<128>, sizeof(DqSmem<128>) + 1024, grid_dq, 384, a, dqm, s,

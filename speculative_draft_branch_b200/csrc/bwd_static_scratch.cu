@@ -5,14 +5,15 @@
 // pool at start-up, or a plugin whose host forbids allocation once it is
 // running.  Such callers cannot cudaMalloc the backward workspace that
 // branch_attn_bwd asks for.  This entry point runs the same backward with its
-// scratch (D = rowsum(dO * O) and the fp32 dQ accumulator) placed in a
-// file-scope device array instead, so it allocates nothing.
+// scratch (D = rowsum(dO * O) plus the fp32 dQ accumulator or the per-query
+// records) placed in a file-scope device array instead, so it allocates
+// nothing.
 //
 // The array is a module global: every GPU that loads this library holds
 // kStaticScratchBytes of it until the process exits.  All calls on a device
 // share that one array and it keeps whatever the last call left in it; the
-// backward zeroes the dQ accumulator and overwrites D itself on every call,
-// so nothing has to be cleared in between.  Two calls whose kernels overlap on
+// backward rewrites D and the records (or zeroes the dQ accumulator) itself on
+// every call, so nothing has to be cleared in between.  Two calls whose kernels overlap on
 // the GPU (different streams without ordering) race on the array.
 #include <mutex>
 
