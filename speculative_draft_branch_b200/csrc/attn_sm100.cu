@@ -204,11 +204,11 @@ __global__ void __launch_bounds__(256, 1)
           !mbar_wait(smem_u32(&sm.bar_p_full[pb]), (i >> 1) & 1, abort_flag, status_word, 4))
         return false;
       tc_fence_after();
-      const uint32_t v_s = smem_u32(sm.v[st]);
+      const uint64_t vd = sdesc(smem_u32(sm.v[st]), 16384, 1024);
       // O += P V: P (bf16 pairs) from TMEM, V as an MN-major operand
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        mma_bf16_ts(t_o, t_p(pb) + k * 8, sdesc(v_s + k * 2048, 16384, 1024), idesc_pv,
+        mma_bf16_ts(t_o, t_p(pb) + k * 8, desc_at(vd, k * 2048), idesc_pv,
                     (i > 0 || k > 0) ? 1u : 0u);
       mma_commit(b_o);
       mma_commit(smem_u32(&sm.bar_v_empty[st]));
@@ -224,12 +224,11 @@ __global__ void __launch_bounds__(256, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t k_s = smem_u32(sm.k[st]);
+      const uint64_t qd = sdesc(q_s, 16, 1024), kd = sdesc(smem_u32(sm.k[st]), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-        mma_bf16(tmem + sb * 128, sdesc(q_s + off, 16, 1024), sdesc(k_s + off, 16, 1024),
-                 idesc_qk, k > 0 ? 1u : 0u);
+        mma_bf16(tmem + sb * 128, desc_at(qd, off), desc_at(kd, off), idesc_qk, k > 0 ? 1u : 0u);
       }
       mma_commit(smem_u32(&sm.bar_s_full[sb]));
       mma_commit(smem_u32(&sm.bar_k_empty[st]));
@@ -580,12 +579,12 @@ __global__ void __launch_bounds__(384, 1)
           !mbar_wait(smem_u32(&sm.bar_k_full[st]), (j / kFwd2Stages) & 1, abort_flag, status_word, 5))
         return false;
       tc_fence_after();
-      const uint32_t q_s = smem_u32(sm.q[x]), k_s = smem_u32(sm.k[st]);
+      const uint64_t qd = sdesc(smem_u32(sm.q[x]), 16, 1024);
+      const uint64_t kd = sdesc(smem_u32(sm.k[st]), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-        mma_bf16(t_s(x), sdesc(q_s + off, 16, 1024), sdesc(k_s + off, 16, 1024), idesc_qk,
-                 k > 0 ? 1u : 0u);
+        mma_bf16(t_s(x), desc_at(qd, off), desc_at(kd, off), idesc_qk, k > 0 ? 1u : 0u);
       }
       mma_commit(smem_u32(&sm.bar_s_full[x]));
       if (x == 1) mma_commit(smem_u32(&sm.bar_k_empty[st]));
@@ -598,10 +597,10 @@ __global__ void __launch_bounds__(384, 1)
           !mbar_wait(smem_u32(&sm.bar_p_full[x]), i & 1, abort_flag, status_word, 4))
         return false;
       tc_fence_after();
-      const uint32_t v_s = smem_u32(sm.v[st]);
+      const uint64_t vd = sdesc(smem_u32(sm.v[st]), 16384, 1024);
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        mma_bf16_ts(t_o(x), t_s(x) + k * 8, sdesc(v_s + k * 2048, 16384, 1024), idesc_pv,
+        mma_bf16_ts(t_o(x), t_s(x) + k * 8, desc_at(vd, k * 2048), idesc_pv,
                     (i > 0 || k > 0) ? 1u : 0u);
       if (x == 1) mma_commit(smem_u32(&sm.bar_v_empty[st]));
       return true;

@@ -167,16 +167,16 @@ __global__ void __launch_bounds__(384, 1)
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
     constexpr uint32_t idesc_dq = idesc_bf16(128, D, false, true);
     bool ok = total == 0 || mbar_wait(b_qdo, 0, abort_flag, status_word, 3);
-    const uint32_t q_s = smem_u32(sm.q), do_s = smem_u32(sm.dout);
+    const uint64_t qd0 = sdesc(smem_u32(sm.q), 16, 1024), dod0 = sdesc(smem_u32(sm.dout), 16, 1024);
     auto issue_dq = [&](int i) -> bool {
       if (!mbar_wait(smem_u32(&sm.bar_ds_full[i & 1]), (i >> 1) & 1, abort_flag, status_word, 4))
         return false;
       tc_fence_after();
-      const uint32_t k_s = smem_u32(sm.k[i % kDqKStages]);
+      const uint64_t kd = sdesc(smem_u32(sm.k[i % kDqKStages]), 16384, 1024);
       // dQ += dS K: dS (bf16 pairs) from TMEM, K as an MN-major operand
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        mma_bf16_ts(t_dq, t_ds(i & 1) + k * 8, sdesc(k_s + k * 2048, 16384, 1024), idesc_dq,
+        mma_bf16_ts(t_dq, t_ds(i & 1) + k * 8, desc_at(kd, k * 2048), idesc_dq,
                     (i > 0 || k > 0) ? 1u : 0u);
       mma_commit(smem_u32(&sm.bar_k_empty[i % kDqKStages]));
       return true;
@@ -192,18 +192,17 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t k_s = smem_u32(sm.k[ks]), v_s = smem_u32(sm.v[vs]);
+      const uint64_t kd = sdesc(smem_u32(sm.k[ks]), 16, 1024);
+      const uint64_t vd = sdesc(smem_u32(sm.v[vs]), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-        mma_bf16(t_s, sdesc(q_s + off, 16, 1024), sdesc(k_s + off, 16, 1024), idesc_s,
-                 k > 0 ? 1u : 0u);
+        mma_bf16(t_s, desc_at(qd0, off), desc_at(kd, off), idesc_s, k > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-        mma_bf16(t_dp, sdesc(do_s + off, 16, 1024), sdesc(v_s + off, 16, 1024), idesc_s,
-                 k > 0 ? 1u : 0u);
+        mma_bf16(t_dp, desc_at(dod0, off), desc_at(vd, off), idesc_s, k > 0 ? 1u : 0u);
       }
       mma_commit(b_sdp_full);
       mma_commit(smem_u32(&sm.bar_v_empty[vs]));
@@ -461,22 +460,23 @@ __global__ void __launch_bounds__(384, 1)
     constexpr uint32_t idesc_s = idesc_bf16(128, kQc, false, false);
     constexpr uint32_t idesc_g = idesc_bf16(128, D, false, true);
     bool ok = total == 0 || mbar_wait(b_kv, 0, abort_flag, status_word, 3);
-    const uint32_t k_s = smem_u32(sm.k), v_s = smem_u32(sm.v);
+    const uint64_t kd0 = sdesc(smem_u32(sm.k), 16, 1024), vd0 = sdesc(smem_u32(sm.v), 16, 1024);
     auto grads = [&](int i) -> bool {
       const int sb = i & 1, st = i % kKvStages;
       if (!mbar_wait(smem_u32(&sm.bar_pds_full[sb]), (i >> 1) & 1, abort_flag, status_word, 4))
         return false;
       tc_fence_after();
-      const uint32_t q_s = smem_u32(sm.q[st]), do_s = smem_u32(sm.dout[st]);
+      const uint64_t qd = sdesc(smem_u32(sm.q[st]), 8192, 1024);
+      const uint64_t dod = sdesc(smem_u32(sm.dout[st]), 8192, 1024);
       // dV += P^T dO, dK += dS^T Q (P^T, dS^T from TMEM; K = 64 queries)
 #pragma unroll
       for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16_ts(t_dv, t_s(sb) + (k >> 1) * 32 + (k & 1) * 8,
-                    sdesc(do_s + k * 2048, 8192, 1024), idesc_g, (i > 0 || k > 0) ? 1u : 0u);
+        mma_bf16_ts(t_dv, t_s(sb) + (k >> 1) * 32 + (k & 1) * 8, desc_at(dod, k * 2048), idesc_g,
+                    (i > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
       for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16_ts(t_dk, t_dp(sb) + (k >> 1) * 32 + (k & 1) * 8,
-                    sdesc(q_s + k * 2048, 8192, 1024), idesc_g, (i > 0 || k > 0) ? 1u : 0u);
+        mma_bf16_ts(t_dk, t_dp(sb) + (k >> 1) * 32 + (k & 1) * 8, desc_at(qd, k * 2048), idesc_g,
+                    (i > 0 || k > 0) ? 1u : 0u);
       mma_commit(smem_u32(&sm.bar_qdo_empty[st]));
       return true;
     };
@@ -490,20 +490,19 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       // S^T / dP^T buffer sb was last read (as P^T / dS^T) by grads(c - 2),
       // issued before this point: tcgen05 MMAs of one thread run in order
-      const uint32_t q_s = smem_u32(sm.q[st]), do_s = smem_u32(sm.dout[st]);
+      const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16, 1024);
+      const uint64_t dod = sdesc(smem_u32(sm.dout[st]), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
         const uint32_t qa = (k >> 2) * 8192 + (k & 3) * 32;
-        mma_bf16(t_s(sb), sdesc(k_s + ka, 16, 1024), sdesc(q_s + qa, 16, 1024), idesc_s,
-                 k > 0 ? 1u : 0u);
+        mma_bf16(t_s(sb), desc_at(kd0, ka), desc_at(qd, qa), idesc_s, k > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
         const uint32_t qa = (k >> 2) * 8192 + (k & 3) * 32;
-        mma_bf16(t_dp(sb), sdesc(v_s + ka, 16, 1024), sdesc(do_s + qa, 16, 1024), idesc_s,
-                 k > 0 ? 1u : 0u);
+        mma_bf16(t_dp(sb), desc_at(vd0, ka), desc_at(dod, qa), idesc_s, k > 0 ? 1u : 0u);
       }
       mma_commit(smem_u32(&sm.bar_sdp_full[sb]));
       if (c >= 1 && !grads(c - 1)) {

@@ -207,6 +207,14 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes,
   return d;
 }
 
+// Descriptor of the same operand `bytes` further on: the start address is the
+// low 14-bit field (address >> 4) and shared-memory addresses stay below
+// 256 KB, so the add never carries out of the field.  Lets an MMA loop build
+// one descriptor per operand and step it with constants.
+__device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B.
 //   bits 4-5 D format (1 = f32)   bits 7-9 A format (1 = bf16)
 //   bits 10-12 B format (1 = bf16)   bit 15 A MN-major   bit 16 B MN-major
