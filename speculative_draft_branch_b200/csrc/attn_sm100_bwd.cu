@@ -18,13 +18,15 @@
 //                      rings so V is refilled as soon as dP is done.
 //   dkdv_sm100_kernel  key-stationary (one CTA per 128-row key tile and kv
 //                      head, the plan's backward work order): over every
-//                      64-row query chunk of every q head of the group that
+//                      128-row query tile of every q head of the group that
 //                      visits the tile, S^T = K Q^T and dP^T = V dO^T into
-//                      double-buffered TMEM, P^T and dS^T written over them as
-//                      bf16, dV += P^T dO and dK += dS^T Q (A operands from
-//                      TMEM) accumulated in TMEM for the whole walk.  Per-query
-//                      records {LSE, D, key interval} arrive by bulk copy with
-//                      the Q / dO tiles through a 4-deep ring.
+//                      TMEM (N = 128: the tensor cores' full rate), P^T and
+//                      dS^T written over dP^T as bf16, dV += P^T dO and
+//                      dK += dS^T Q (A operands from TMEM) accumulated in TMEM
+//                      for the whole walk.  Q and dO come through separate
+//                      two-deep rings, each freed by the product that reads it
+//                      last; per-query records {LSE, D, key interval} arrive by
+//                      bulk copy with dO.
 #include "attn_sm100_common.cuh"
 
 namespace ba {
@@ -314,19 +316,21 @@ __global__ void __launch_bounds__(384, 1)
 // ============================================================================
 // dK / dV kernel
 // ============================================================================
-constexpr int kQc = 64;      // query rows per chunk
-constexpr int kKvStages = 4;  // Q / dO / record ring depth
+constexpr int kQc = 128;      // query rows per chunk: N of the S^T / dP^T products
+constexpr int kQStages = 2;   // Q ring (freed once dK of the chunk is done)
+constexpr int kDoStages = 2;  // dO + records ring (freed once dV of the chunk is done)
 
 template <int D>
 struct DkvSmem {
   bf16 k[128 * D];
   bf16 v[128 * D];
-  bf16 q[kKvStages][kQc * D];     // D/64 boxes of [64 rows][64], 8 KB each
-  bf16 dout[kKvStages][kQc * D];
-  float4 rec[kKvStages][kQc];     // {LSE log2, D, key lo, key hi} per query
+  bf16 q[kQStages][kQc * D];      // D/64 boxes of [128 rows][64], 16 KB each
+  bf16 dout[kDoStages][kQc * D];
+  float4 rec[kDoStages][kQc];     // {LSE log2, D, key lo, key hi} per query
   uint64_t bar_kv;
-  uint64_t bar_qdo_full[kKvStages], bar_qdo_empty[kKvStages];
-  uint64_t bar_sdp_full[2], bar_pds_full[2];
+  uint64_t bar_q_full[kQStages], bar_q_empty[kQStages];
+  uint64_t bar_do_full[kDoStages], bar_do_empty[kDoStages];
+  uint64_t bar_s_full, bar_x_free, bar_dp_full, bar_pds_full;
   uint64_t bar_acc_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -334,29 +338,39 @@ struct DkvSmem {
 
 struct DkvMaps {
   TensorMaps t;
-  CUtensorMap q64_m, q64_b, do64_m, do64_b;  // 64-row boxes
+  CUtensorMap do_m, do_b;
 };
 
+// Chunk c of a CTA's walk: query tile step s = c / grp, q head g grp + c % grp.
+// The tile steps merge the CTA's main q tiles and branch q tiles, each taken
+// from the last down, interleaved in proportion to their counts.  Every CTA
+// of a sequence then starts on the same (highest) tiles and moves through
+// them at the same pace, so the Q / dO tiles one CTA loads are still in L2
+// when the CTAs of the other key tiles of that sequence ask for them.
 struct ChunkWalk {
-  int n_t0, n_t1, t0, t1, per_head, grp, g;
+  int n_t0, n_t1, t0, t1, grp, g;
   __device__ __forceinline__ void at(int c, const AttnParams &a, int &h, bool &is_main_q,
-                                     int &tile, int &row0, int &nrows) const {
-    const int hh = c / per_head, rem = c % per_head;
-    const int ti = rem >> 1, half = rem & 1;
-    h = g * grp + hh;
-    is_main_q = ti < n_t0;
-    tile = is_main_q ? t0 + ti : t1 + (ti - n_t0);
+                                     int &tile, int &nrows) const {
+    const int s = c / grp;
+    h = g * grp + (c - s * grp);
+    const int n = n_t0 + n_t1;
+    const int m0 = (int)((int64_t)s * n_t0 / n);
+    const int m1 = (int)((int64_t)(s + 1) * n_t0 / n);
+    is_main_q = m1 > m0;
+    tile = is_main_q ? t0 + n_t0 - 1 - m0 : t1 + n_t1 - 1 - (s - m0);
     const int rows = is_main_q ? a.n_main : a.n_bt;
-    row0 = tile * 128 + half * kQc;
-    nrows = max(0, min(kQc, rows - row0));
+    nrows = max(0, min(kQc, rows - tile * kQc));
   }
 };
 
-// TMEM columns: dK [0, 128), dV [128, 256), S^T / P^T buffers at 256 and 320,
-// dP^T / dS^T buffers at 384 and 448.  Two threads per key row: the thread for
-// queries [32h, 32h + 32) writes their P^T / dS^T (bf16 pairs) over columns
-// [32h, 32h + 16) of the S^T / dP^T it read, so K-step k (16 queries) of the
-// dV / dK products sits at column (k / 2) * 32 + (k % 2) * 8.
+// TMEM columns: dK [0, D), dV [D, 2D), X = S^T at 2D, Y = dP^T at 2D + 128
+// (128 columns each).  Two threads per key row, one per query half
+// [64 qh, 64 qh + 64): each reads its S^T half from X (freeing X for the next
+// chunk's S^T as soon as every thread has it in registers), then, 32 queries
+// at a time, reads dP^T from Y and writes P^T and dS^T (bf16 pairs, 16
+// columns each) over the 32 columns it read.  K-step k (queries 16k..16k+15)
+// of the dV product reads P^T at Y + 32 (k / 2) + 8 (k % 2), that of the dK
+// product dS^T 16 columns further.
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     dkdv_sm100_kernel(const AttnParams a, const __grid_constant__ DkvMaps tm) {
@@ -382,22 +396,27 @@ __global__ void __launch_bounds__(384, 1)
     const int32_t *r = a.plan.kv_branch + (int64_t)kt * 2;
     cw.t0 = 0; cw.n_t0 = 0; cw.t1 = r[0]; cw.n_t1 = r[1] - r[0];
   }
-  cw.per_head = 2 * (cw.n_t0 + cw.n_t1);
-  const int total = cw.grp * cw.per_head;
+  const int total = cw.grp * (cw.n_t0 + cw.n_t1);
   int *status_word = a.plan.status + 1;
   volatile int *abort_flag = &sm.abort_flag;
 
   const uint32_t b_kv = smem_u32(&sm.bar_kv), b_acc = smem_u32(&sm.bar_acc_done);
+  const uint32_t b_s = smem_u32(&sm.bar_s_full), b_xf = smem_u32(&sm.bar_x_free);
+  const uint32_t b_dp = smem_u32(&sm.bar_dp_full), b_pds = smem_u32(&sm.bar_pds_full);
   if (threadIdx.x == 0) {
     mbar_init(b_kv, 1);
-    for (int s = 0; s < kKvStages; ++s) {
-      mbar_init(smem_u32(&sm.bar_qdo_full[s]), 1);
-      mbar_init(smem_u32(&sm.bar_qdo_empty[s]), 1);
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(smem_u32(&sm.bar_q_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_q_empty[s]), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&sm.bar_sdp_full[s]), 1);
-      mbar_init(smem_u32(&sm.bar_pds_full[s]), 256);
+    for (int s = 0; s < kDoStages; ++s) {
+      mbar_init(smem_u32(&sm.bar_do_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_do_empty[s]), 1);
     }
+    mbar_init(b_s, 1);
+    mbar_init(b_xf, 256);
+    mbar_init(b_dp, 1);
+    mbar_init(b_pds, 256);
     mbar_init(b_acc, 1);
     sm.abort_flag = 0;
     mbar_fence_init();
@@ -410,9 +429,7 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t t_dk = tmem, t_dv = tmem + 128;
-  auto t_s = [&](int b) { return tmem + 256 + b * 64; };
-  auto t_dp = [&](int b) { return tmem + 384 + b * 64; };
+  const uint32_t t_dk = tmem, t_dv = tmem + D, t_x = tmem + 2 * D, t_y = tmem + 2 * D + 128;
   // records of this CTA's key kind: main-key intervals or branch-local ones
   const float4 *rec_base = a.rec + (main_kv ? 0 : (int64_t)a.hq * a.rows_pad);
 
@@ -428,150 +445,189 @@ __global__ void __launch_bounds__(384, 1)
         tma_load_3d(smem_u32(sm.v) + x * 16384, vm, b_kv, x * 64, g, key0);
       }
     }
-    int issued = 0;
+    int q_issued = 0, do_issued = 0;
     for (int c = 0; c < total; ++c) {
-      const int st = c % kKvStages;
-      if (c >= kKvStages &&
-          !mbar_wait(smem_u32(&sm.bar_qdo_empty[st]), ((c / kKvStages) - 1) & 1, abort_flag,
+      int h, tile, nrows;
+      bool is_main_q;
+      cw.at(c, a, h, is_main_q, tile, nrows);
+      const int row0 = tile * kQc;
+      const int st = c % kQStages, ds = c % kDoStages;
+      if (c >= kQStages &&
+          !mbar_wait(smem_u32(&sm.bar_q_empty[st]), ((c / kQStages) - 1) & 1, abort_flag,
                      status_word, 1))
         break;
-      int h, tile, row0, nrows;
-      bool is_main_q;
-      cw.at(c, a, h, is_main_q, tile, row0, nrows);
-      const uint32_t bar = smem_u32(&sm.bar_qdo_full[st]);
-      mbar_expect_tx(bar, 2 * kQc * D * 2 + kQc * 16);
-      const CUtensorMap *qm = is_main_q ? &tm.q64_m : &tm.q64_b;
-      const CUtensorMap *dm = is_main_q ? &tm.do64_m : &tm.do64_b;
+      const uint32_t qbar = smem_u32(&sm.bar_q_full[st]);
+      mbar_expect_tx(qbar, kQc * D * 2);
+      const CUtensorMap *qm = is_main_q ? &tm.t.q_m : &tm.t.q_b;
 #pragma unroll
-      for (int x = 0; x < D / 64; ++x) {
-        tma_load_3d(smem_u32(sm.q[st]) + x * 8192, qm, bar, x * 64, h, row0);
-        tma_load_3d(smem_u32(sm.dout[st]) + x * 8192, dm, bar, x * 64, h, row0);
-      }
+      for (int x = 0; x < D / 64; ++x)
+        tma_load_3d(smem_u32(sm.q[st]) + x * 16384, qm, qbar, x * 64, h, row0);
+      ++q_issued;
+      if (c >= kDoStages &&
+          !mbar_wait(smem_u32(&sm.bar_do_empty[ds]), ((c / kDoStages) - 1) & 1, abort_flag,
+                     status_word, 1))
+        break;
+      const uint32_t dbar = smem_u32(&sm.bar_do_full[ds]);
+      mbar_expect_tx(dbar, kQc * D * 2 + kQc * 16);
+      const CUtensorMap *dm = is_main_q ? &tm.do_m : &tm.do_b;
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x)
+        tma_load_3d(smem_u32(sm.dout[ds]) + x * 16384, dm, dbar, x * 64, h, row0);
       const int64_t prow = (is_main_q ? 0 : a.n_main_pad) + row0;
-      bulk_load(smem_u32(sm.rec[st]), rec_base + (int64_t)h * a.rows_pad + prow, kQc * 16, bar);
-      ++issued;
+      bulk_load(smem_u32(sm.rec[ds]), rec_base + (int64_t)h * a.rows_pad + prow, kQc * 16, dbar);
+      ++do_issued;
     }
-    for (int c = (issued > kKvStages ? issued - kKvStages : 0); c < issued; ++c)
-      mbar_wait(smem_u32(&sm.bar_qdo_full[c % kKvStages]), (c / kKvStages) & 1, abort_flag,
+    // no copy may still be writing shared memory when the CTA exits
+    for (int c = (q_issued > kQStages ? q_issued - kQStages : 0); c < q_issued; ++c)
+      mbar_wait(smem_u32(&sm.bar_q_full[c % kQStages]), (c / kQStages) & 1, abort_flag,
+                status_word, 2);
+    for (int c = (do_issued > kDoStages ? do_issued - kDoStages : 0); c < do_issued; ++c)
+      mbar_wait(smem_u32(&sm.bar_do_full[c % kDoStages]), (c / kDoStages) & 1, abort_flag,
                 status_word, 2);
     if (total > 0) mbar_wait(b_kv, 0, abort_flag, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order per chunk c: S^T(c+1), dK(c), dV(c), dP^T(c+1).  S^T(c+1)
+    // overwrites X once the P^T threads hold S^T(c); dP^T(c+1) overwrites Y
+    // after dK(c) / dV(c) have read P^T and dS^T from it: tcgen05 MMAs issued
+    // by one thread run in order.
     constexpr uint32_t idesc_s = idesc_bf16(128, kQc, false, false);
     constexpr uint32_t idesc_g = idesc_bf16(128, D, false, true);
     bool ok = total == 0 || mbar_wait(b_kv, 0, abort_flag, status_word, 3);
     const uint64_t kd0 = sdesc(smem_u32(sm.k), 16, 1024), vd0 = sdesc(smem_u32(sm.v), 16, 1024);
-    auto grads = [&](int i) -> bool {
-      const int sb = i & 1, st = i % kKvStages;
-      if (!mbar_wait(smem_u32(&sm.bar_pds_full[sb]), (i >> 1) & 1, abort_flag, status_word, 4))
+    auto issue_s = [&](int c) -> bool {
+      const int st = c % kQStages;
+      if (!mbar_wait(smem_u32(&sm.bar_q_full[st]), (c / kQStages) & 1, abort_flag, status_word,
+                     5))
         return false;
+      if (c > 0 && !mbar_wait(b_xf, (c - 1) & 1, abort_flag, status_word, 6)) return false;
       tc_fence_after();
-      const uint64_t qd = sdesc(smem_u32(sm.q[st]), 8192, 1024);
-      const uint64_t dod = sdesc(smem_u32(sm.dout[st]), 8192, 1024);
-      // dV += P^T dO, dK += dS^T Q (P^T, dS^T from TMEM; K = 64 queries)
+      const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16, 1024);
 #pragma unroll
-      for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16_ts(t_dv, t_s(sb) + (k >> 1) * 32 + (k & 1) * 8, desc_at(dod, k * 2048), idesc_g,
-                    (i > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-      for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16_ts(t_dk, t_dp(sb) + (k >> 1) * 32 + (k & 1) * 8, desc_at(qd, k * 2048), idesc_g,
-                    (i > 0 || k > 0) ? 1u : 0u);
-      mma_commit(smem_u32(&sm.bar_qdo_empty[st]));
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+        mma_bf16(t_x, desc_at(kd0, off), desc_at(qd, off), idesc_s, k > 0 ? 1u : 0u);
+      }
+      mma_commit(b_s);
       return true;
     };
-    for (int c = 0; ok && c < total; ++c) {
-      const int st = c % kKvStages, sb = c & 1;
-      if (!mbar_wait(smem_u32(&sm.bar_qdo_full[st]), (c / kKvStages) & 1, abort_flag, status_word,
-                     5)) {
-        ok = false;
-        break;
-      }
+    auto issue_dp = [&](int c) -> bool {
+      const int ds = c % kDoStages;
+      if (!mbar_wait(smem_u32(&sm.bar_do_full[ds]), (c / kDoStages) & 1, abort_flag, status_word,
+                     5))
+        return false;
       tc_fence_after();
-      // S^T / dP^T buffer sb was last read (as P^T / dS^T) by grads(c - 2),
-      // issued before this point: tcgen05 MMAs of one thread run in order
-      const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16, 1024);
-      const uint64_t dod = sdesc(smem_u32(sm.dout[st]), 16, 1024);
+      const uint64_t dd = sdesc(smem_u32(sm.dout[ds]), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
-        const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
-        const uint32_t qa = (k >> 2) * 8192 + (k & 3) * 32;
-        mma_bf16(t_s(sb), desc_at(kd0, ka), desc_at(qd, qa), idesc_s, k > 0 ? 1u : 0u);
+        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+        mma_bf16(t_y, desc_at(vd0, off), desc_at(dd, off), idesc_s, k > 0 ? 1u : 0u);
       }
+      mma_commit(b_dp);
+      return true;
+    };
+    auto issue_grads = [&](int c) -> bool {
+      if (!mbar_wait(b_pds, c & 1, abort_flag, status_word, 4)) return false;
+      tc_fence_after();
+      const int st = c % kQStages, ds = c % kDoStages;
+      // B operands MN-major: K = 16 queries per step (16 rows of 128 B), the
+      // two 64-column halves of D one 16 KB box apart
+      const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16384, 1024);
+      const uint64_t dd = sdesc(smem_u32(sm.dout[ds]), 16384, 1024);
+      // dK += dS^T Q, then dV += P^T dO (K = 128 queries)
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t ka = (k >> 2) * 16384 + (k & 3) * 32;
-        const uint32_t qa = (k >> 2) * 8192 + (k & 3) * 32;
-        mma_bf16(t_dp(sb), desc_at(vd0, ka), desc_at(dod, qa), idesc_s, k > 0 ? 1u : 0u);
-      }
-      mma_commit(smem_u32(&sm.bar_sdp_full[sb]));
-      if (c >= 1 && !grads(c - 1)) {
-        ok = false;
-        break;
-      }
+      for (int k = 0; k < kQc / 16; ++k)
+        mma_bf16_ts(t_dk, t_y + (k >> 1) * 32 + 16 + (k & 1) * 8, desc_at(qd, k * 2048), idesc_g,
+                    (c > 0 || k > 0) ? 1u : 0u);
+      mma_commit(smem_u32(&sm.bar_q_empty[st]));
+#pragma unroll
+      for (int k = 0; k < kQc / 16; ++k)
+        mma_bf16_ts(t_dv, t_y + (k >> 1) * 32 + (k & 1) * 8, desc_at(dd, k * 2048), idesc_g,
+                    (c > 0 || k > 0) ? 1u : 0u);
+      mma_commit(smem_u32(&sm.bar_do_empty[ds]));
+      return true;
+    };
+    if (ok && total > 0) ok = issue_s(0) && issue_dp(0);
+    for (int c = 0; ok && c < total; ++c) {
+      if (c + 1 < total && !issue_s(c + 1)) ok = false;
+      else if (!issue_grads(c)) ok = false;
+      else if (c + 1 < total && !issue_dp(c + 1)) ok = false;
     }
-    if (ok && total > 0 && grads(total - 1)) mma_commit(b_acc);
+    if (ok && total > 0) mma_commit(b_acc);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ P^T, dS^T (2 threads / key)
     const int ew = threadIdx.x - 128;
-    const int qh = ew >> 7;           // query half: [32 qh, 32 qh + 32)
+    const int qh = ew >> 7;           // query half: [64 qh, 64 qh + 64)
     const int row = ew & 127;
     const int key = key0 + row;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
     bool ok = true;
     for (int c = 0; c < total; ++c) {
-      const int st = c % kKvStages, sb = c & 1;
+      const int ds = c % kDoStages;
       // a chunk whose every query sees every key of this tile needs no mask
       bool full = false;
       if (main_kv) {
-        int h, tile, row0, nrows;
+        int h, tile, nrows;
         bool is_main_q;
-        cw.at(c, a, h, is_main_q, tile, row0, nrows);
+        cw.at(c, a, h, is_main_q, tile, nrows);
         const int32_t *qt =
             a.plan.qtile + (int64_t)(is_main_q ? tile : a.n_qt_main + tile) * 6;
         full = nrows == kQc && kt >= qt[1] && kt < qt[2];
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_sdp_full[sb]), (c >> 1) & 1,
-                                             abort_flag, status_word, 7)) ||
-          !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_qdo_full[st]),
-                                             (c / kKvStages) & 1, abort_flag, status_word, 8))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(b_s, c & 1, abort_flag, status_word, 7))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[32], dp[32];
-      tmem_ld32(t_s(sb) + lane_addr + qh * 32, reinterpret_cast<uint32_t *>(s));
-      tmem_ld32(t_dp(sb) + lane_addr + qh * 32, reinterpret_cast<uint32_t *>(dp));
+      float p[64];
+      tmem_ld32(t_x + lane_addr + qh * 64, reinterpret_cast<uint32_t *>(p));
+      tmem_ld32(t_x + lane_addr + qh * 64 + 32, reinterpret_cast<uint32_t *>(p + 32));
       tc_wait_ld();
-      const float4 *rec = sm.rec[st] + qh * 32;
+      tc_fence_before();
+      mbar_arrive(b_xf);
+      // the records come with dO
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_do_full[ds]), (c / kDoStages) & 1,
+                                             abort_flag, status_word, 8))) {
+        ok = false;
+        break;
+      }
+      const float4 *rec = sm.rec[ds] + qh * 64;
       if (!full) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < 64; ++q) {
           const int2 iv =
               *reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(&rec[q]) + 8);
-          if (key < iv.x || key > iv.y) s[q] = kNegInf;
+          if (key < iv.x || key > iv.y) p[q] = kNegInf;
         }
       }
-      uint32_t pk[16], dk2[16];
 #pragma unroll
-      for (int q = 0; q < 32; q += 2) {
-        float p2[2], d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float2 r = *reinterpret_cast<const float2 *>(&rec[q + e]);
-          const float p = ex2(fmaf(s[q + e], sl2, -r.x));
-          p2[e] = p;
-          d2[e] = p * (dp[q + e] - r.y);
-        }
-        pk[q / 2] = pack_bf16(p2[0], p2[1]);
-        dk2[q / 2] = pack_bf16(d2[0], d2[1]);
+      for (int q = 0; q < 64; ++q) p[q] = ex2(fmaf(p[q], sl2, -rec[q].x));
+      if (!__all_sync(0xffffffffu, mbar_wait(b_dp, c & 1, abort_flag, status_word, 9))) {
+        ok = false;
+        break;
       }
-      tmem_st16(t_s(sb) + lane_addr + qh * 32, pk);
-      tmem_st16(t_dp(sb) + lane_addr + qh * 32, dk2);
+      tc_fence_after();
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const uint32_t col = t_y + lane_addr + qh * 64 + pass * 32;
+        float dp[32];
+        tmem_ld32(col, reinterpret_cast<uint32_t *>(dp));
+        tc_wait_ld();
+        uint32_t pk[16], dk2[16];
+#pragma unroll
+        for (int q = 0; q < 32; q += 2) {
+          const float p0 = p[pass * 32 + q], p1 = p[pass * 32 + q + 1];
+          pk[q / 2] = pack_bf16(p0, p1);
+          dk2[q / 2] = pack_bf16(p0 * (dp[q] - rec[pass * 32 + q].y),
+                                 p1 * (dp[q + 1] - rec[pass * 32 + q + 1].y));
+        }
+        tmem_st16(col, pk);
+        tmem_st16(col + 16, dk2);
+      }
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.bar_pds_full[sb]));
+      mbar_arrive(b_pds);
     }
     if (ok && total > 0 &&
         !__all_sync(0xffffffffu, mbar_wait(b_acc, 0, abort_flag, status_word, 10)))
@@ -654,14 +710,8 @@ ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s) {
   if (br) { BA_MAP(dqm.do_b, a.do_b, a.n_bt, a.hq, 128) } else { dqm.do_b = dqm.do_m; }
   DkvMaps kvm;
   kvm.t = t;
-  BA_MAP(kvm.q64_m, a.q_m, a.n_main, a.hq, kQc)
-  BA_MAP(kvm.do64_m, a.do_m, a.n_main, a.hq, kQc)
-  if (br) {
-    BA_MAP(kvm.q64_b, a.q_b, a.n_bt, a.hq, kQc)
-    BA_MAP(kvm.do64_b, a.do_b, a.n_bt, a.hq, kQc)
-  } else {
-    kvm.q64_b = kvm.q64_m; kvm.do64_b = kvm.do64_m;
-  }
+  kvm.do_m = dqm.do_m;
+  kvm.do_b = dqm.do_b;
 #undef BA_MAP
   const int64_t grid_dq = (int64_t)a.n_qt * a.hq;
   const int64_t grid_kv = (int64_t)(a.n_kt + a.n_bkt) * a.hkv;
