@@ -223,6 +223,32 @@ BA_API ba_status branch_attn_bwd_static_scratch(
     const void *do_b, void *dq_m, void *dk_m, void *dv_m, void *dq_b, void *dk_b, void *dv_b,
     ba_stream_t stream);
 
+/* One training step on host buffers (no counterpart in the paper; an
+ * interface addition for callers whose tensors live in host memory).
+ * Copies the metadata and the eight inputs into `staging` (device memory of
+ * at least ba_step_host_workspace_size bytes, owned by the caller), builds
+ * the plan, runs branch_attn_fwd and branch_attn_bwd, and copies O, LSE and
+ * the six gradients back, all enqueued on `stream`; the call returns without
+ * waiting.  Here the metadata pointers of *p (cu_seqlens, branch_anchor,
+ * branch_depth) are HOST pointers, like every tensor argument.  Layouts are
+ * those of branch_attn_fwd / branch_attn_bwd.
+ *   - Copies run on two streams the library keeps per device (one upload,
+ *     one download): dO is uploaded while the forward runs and O / LSE are
+ *     downloaded while the backward runs, and the upload of a step issued on
+ *     another stream (with its own staging) overlaps this step's download.
+ *   - Host buffers should be page-locked; pageable memory works but the
+ *     copies then do not overlap.
+ *   - The host outputs are complete once `stream` reaches the point after
+ *     this call.  Inputs must stay unchanged until then.
+ *   - Plan content errors are not checked here; ba_plan_status on the plan
+ *     inside the staging area (at offset 0) reports them after the step. */
+BA_API ba_status ba_step_host_workspace_size(const ba_problem *p, size_t *bytes);
+BA_API ba_status branch_attn_step_host(
+    const ba_problem *p, void *staging, size_t staging_bytes, const void *q_m,
+    const void *k_m, const void *v_m, const void *q_b, const void *k_b, const void *v_b,
+    const void *do_m, const void *do_b, void *o_m, void *o_b, float *lse_m, float *lse_b,
+    void *dq_m, void *dk_m, void *dv_m, void *dq_b, void *dk_b, void *dv_b, ba_stream_t stream);
+
 /* Standalone online-softmax merge (technical-contribution section):
  *   l = log(e^{l_a} + e^{l_b}),  O = e^{l_a - l} O_a + e^{l_b - l} O_b.
  * O_* are [rows, heads, head_dim] (fp32 when o_is_fp32, else bf16), l_*
@@ -234,12 +260,12 @@ BA_API ba_status lse_merge(int64_t rows, int32_t heads, int32_t head_dim,
                     const void *o_b, const float *lse_b, void *o_out,
                     float *lse_out, ba_stream_t stream);
 
-/* Device self-check of the exponential used by the softmax (no counterpart
- * in the paper).  The forward softmax evaluates part of its 2^x on the FMA
- * pipe with a range-reduced cubic (max relative error 7.5e-5) and the rest on
- * the hardware ex2 unit; this call writes both for n inputs x (device
- * pointers, fp32): y_fma[i] = polynomial 2^x[i], y_hw[i] = ex2.approx(x[i]).
- * Inputs below -125 (and -inf) give y_fma = 0. */
+/* Device self-check of the exponentials available to the softmax (no
+ * counterpart in the paper): the hardware ex2 unit the kernels use, and a
+ * range-reduced cubic on the FMA pipe (max relative error 7.5e-5) kept as an
+ * alternative for offloading the ex2 unit.  Writes both for n inputs x
+ * (device pointers, fp32): y_fma[i] = polynomial 2^x[i],
+ * y_hw[i] = ex2.approx(x[i]).  Inputs below -125 (and -inf) give y_fma = 0. */
 BA_API ba_status ba_exp2_check(const float *x, float *y_fma, float *y_hw, int64_t n,
                                ba_stream_t stream);
 

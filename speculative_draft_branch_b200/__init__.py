@@ -79,6 +79,8 @@ def _load() -> ctypes.CDLL:
         "ba_get_kernel_family": [],
         "ba_set_kernel_events": [I32, VP, VP],
         "ba_exp2_check": [VP, VP, VP, I64, VP],
+        "ba_step_host_workspace_size": [P, ctypes.POINTER(S)],
+        "branch_attn_step_host": [P, VP, S] + [VP] * 18 + [VP],
         "ba_launch_count": [],
         "ba_last_error": [],
         "ba_version": [],
@@ -261,6 +263,55 @@ def branch_attn_bwd_static_scratch(problem: Problem, plan_ws, q_m, k_m, v_m, q_b
         _ptr(k_b), _ptr(v_b), _ptr(o_m), _ptr(o_b), _ptr(lse_m), _ptr(lse_b), _ptr(do_m),
         _ptr(do_b), _ptr(dq_m), _ptr(dk_m), _ptr(dv_m), _ptr(dq_b), _ptr(dk_b), _ptr(dv_b),
         _stream(stream)))
+
+
+def _expect_host(t, shape, dtype, name):
+    if t is None:
+        if 0 in shape:
+            return
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous() or t.is_cuda:
+        raise ValueError(f"{name}: expected contiguous host {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def ba_step_host_workspace_size(problem: Problem) -> int:
+    """Device staging bytes branch_attn_step_host needs for this problem."""
+    n = ctypes.c_size_t()
+    _check(lib.ba_step_host_workspace_size(ctypes.byref(problem.c), ctypes.byref(n)))
+    return n.value
+
+
+def branch_attn_step_host(problem: Problem, staging, q_m, k_m, v_m, q_b, k_b, v_b, do_m, do_b,
+                          o_m, o_b, lse_m, lse_b, dq_m, dk_m, dv_m, dq_b, dk_b, dv_b,
+                          stream=None) -> None:
+    """One fwd+bwd step on host tensors (pinned for overlap): the problem's
+    index arrays and every tensor are on the host, `staging` is a device
+    uint8 buffer of ba_step_host_workspace_size bytes.  Asynchronous on
+    `stream`; the host outputs are final once the stream reaches this point."""
+    import torch
+    sh = problem.shapes()
+    for name, t, like in (("q_m", q_m, "q_m"), ("k_m", k_m, "k_m"), ("v_m", v_m, "v_m"),
+                          ("q_b", q_b, "q_b"), ("k_b", k_b, "k_b"), ("v_b", v_b, "v_b"),
+                          ("do_m", do_m, "q_m"), ("do_b", do_b, "q_b"), ("o_m", o_m, "q_m"),
+                          ("o_b", o_b, "q_b"), ("dq_m", dq_m, "q_m"), ("dk_m", dk_m, "k_m"),
+                          ("dv_m", dv_m, "v_m"), ("dq_b", dq_b, "q_b"), ("dk_b", dk_b, "k_b"),
+                          ("dv_b", dv_b, "v_b")):
+        _expect_host(t, sh[like], torch.bfloat16, name)
+    _expect_host(lse_m, sh["lse_m"], torch.float32, "lse_m")
+    _expect_host(lse_b, sh["lse_b"], torch.float32, "lse_b")
+    for name, t in (("cu_seqlens", problem.cu_seqlens), ("branch_anchor", problem.branch_anchor),
+                    ("branch_depth", problem.branch_depth)):
+        if t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor for branch_attn_step_host")
+    if not staging.is_cuda:
+        raise ValueError("staging must be a device buffer")
+    nbytes = staging.numel() * staging.element_size()
+    _check(lib.branch_attn_step_host(
+        ctypes.byref(problem.c), _ptr(staging), nbytes, _ptr(q_m), _ptr(k_m), _ptr(v_m),
+        _ptr(q_b), _ptr(k_b), _ptr(v_b), _ptr(do_m), _ptr(do_b), _ptr(o_m), _ptr(o_b),
+        _ptr(lse_m), _ptr(lse_b), _ptr(dq_m), _ptr(dk_m), _ptr(dv_m), _ptr(dq_b), _ptr(dk_b),
+        _ptr(dv_b), _stream(stream)))
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, stream=None) -> None:
