@@ -51,6 +51,7 @@ struct DqSmem {
   uint64_t bar_v_full[kDqVStages], bar_v_empty[kDqVStages];
   uint64_t bar_sdp_full, bar_sdp_empty;
   uint64_t bar_ds_full[2];  // one per dS buffer: the dS threads may run a tile ahead
+  uint64_t bar_dq_done[2];  // dQ(i) has read dS buffer i % 2
   uint64_t bar_dq_final;
   uint32_t tmem_base;
   int abort_flag;
@@ -103,6 +104,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(b_sdp_empty, 256);
     mbar_init(smem_u32(&sm.bar_ds_full[0]), 256);
     mbar_init(smem_u32(&sm.bar_ds_full[1]), 256);
+    mbar_init(smem_u32(&sm.bar_dq_done[0]), 1);
+    mbar_init(smem_u32(&sm.bar_dq_done[1]), 1);
     mbar_init(b_final, 1);
     sm.abort_flag = 0;
     mbar_fence_init();
@@ -165,24 +168,16 @@ __global__ void __launch_bounds__(384, 1)
                 status_word, 2);
     if (total > 0) mbar_wait(b_qdo, 0, abort_flag, status_word, 2);
   } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S / dP issuer
+    // Two issuing threads: this one issues S and dP of each key tile, warp 3
+    // the dQ products.  An mbarrier wait holds the thread that executes it
+    // until the MMAs it has queued are done, so one issuer waiting for dS
+    // would keep the next tile's S / dP out of the tensor pipe (and waiting
+    // for the next K / V would hold back dQ); split, each waits only on its
+    // own inputs.
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
-    constexpr uint32_t idesc_dq = idesc_bf16(128, D, false, true);
-    bool ok = total == 0 || mbar_wait(b_qdo, 0, abort_flag, status_word, 3);
     const uint64_t qd0 = sdesc(smem_u32(sm.q), 16, 1024), dod0 = sdesc(smem_u32(sm.dout), 16, 1024);
-    auto issue_dq = [&](int i) -> bool {
-      if (!mbar_wait(smem_u32(&sm.bar_ds_full[i & 1]), (i >> 1) & 1, abort_flag, status_word, 4))
-        return false;
-      tc_fence_after();
-      const uint64_t kd = sdesc(smem_u32(sm.k[i % kDqKStages]), 16384, 1024);
-      // dQ += dS K: dS (bf16 pairs) from TMEM, K as an MN-major operand
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        mma_bf16_ts(t_dq, t_ds(i & 1) + k * 8, desc_at(kd, k * 2048), idesc_dq,
-                    (i > 0 || k > 0) ? 1u : 0u);
-      mma_commit(smem_u32(&sm.bar_k_empty[i % kDqKStages]));
-      return true;
-    };
+    bool ok = total == 0 || mbar_wait(b_qdo, 0, abort_flag, status_word, 3);
     for (int j = 0; ok && j < total; ++j) {
       const int ks = j % kDqKStages, vs = j % kDqVStages;
       if (!mbar_wait(smem_u32(&sm.bar_k_full[ks]), (j / kDqKStages) & 1, abort_flag, status_word,
@@ -208,12 +203,28 @@ __global__ void __launch_bounds__(384, 1)
       }
       mma_commit(b_sdp_full);
       mma_commit(smem_u32(&sm.bar_v_empty[vs]));
-      if (j >= 1 && !issue_dq(j - 1)) {
+    }
+  } else if (warp == 3 && lane == 0) {
+    // ------------------------------------------------------------ dQ issuer
+    // dQ(i) += dS(i) K(i).  K(i) is released here: S(i) read it before the
+    // dS threads could finish tile i.
+    constexpr uint32_t idesc_dq = idesc_bf16(128, D, false, true);
+    bool ok = true;
+    for (int i = 0; ok && i < total; ++i) {
+      if (!mbar_wait(smem_u32(&sm.bar_ds_full[i & 1]), (i >> 1) & 1, abort_flag, status_word, 4)) {
         ok = false;
         break;
       }
+      tc_fence_after();
+      const uint64_t kd = sdesc(smem_u32(sm.k[i % kDqKStages]), 16384, 1024);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        mma_bf16_ts(t_dq, t_ds(i & 1) + k * 8, desc_at(kd, k * 2048), idesc_dq,
+                    (i > 0 || k > 0) ? 1u : 0u);
+      mma_commit(smem_u32(&sm.bar_k_empty[i % kDqKStages]));
+      mma_commit(smem_u32(&sm.bar_dq_done[i & 1]));
     }
-    if (ok && total > 0 && issue_dq(total - 1)) mma_commit(b_final);
+    if (ok && total > 0) mma_commit(b_final);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ dS (2 threads / row)
     const int ew = threadIdx.x - 128;
@@ -270,7 +281,14 @@ __global__ void __launch_bounds__(384, 1)
         }
         pk[c / 2] = pack_bf16(d2[0], d2[1]);
       }
-      // dS buffer j&1 was last read by dQ_{j-2}, which completed before S_j
+      // dS buffer j&1 was last read by dQ_{j-2}
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_dq_done[j & 1]),
+                                                      ((j - 2) >> 1) & 1, abort_flag,
+                                                      status_word, 8))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
       tmem_st32(t_ds(j & 1) + lane_addr + half * 32, pk);
       tc_wait_st();
       tc_fence_before();
@@ -486,21 +504,25 @@ __global__ void __launch_bounds__(384, 1)
                 status_word, 2);
     if (total > 0) mbar_wait(b_kv, 0, abort_flag, status_word, 2);
   } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
-    // Issue order per chunk c: S^T(c+1), dK(c), dV(c), dP^T(c+1).  S^T(c+1)
-    // overwrites X once the P^T threads hold S^T(c); dP^T(c+1) overwrites Y
-    // after dK(c) / dV(c) have read P^T and dS^T from it: tcgen05 MMAs issued
-    // by one thread run in order.
+    // ------------------------------------------------------------ S^T issuer
+    // Two issuing threads: this one issues S^T(c) = K Q^T into X, warp 3 the
+    // dV / dK products and dP^T(c+1) into Y (in that order: one thread's MMAs
+    // run in order, so dP^T(c+1) overwrites Y only after the gradient
+    // products have read P^T and dS^T from it).  An mbarrier wait holds the
+    // thread that executes it until the MMAs it has queued are done; split,
+    // waiting for the next Q tile no longer holds back the gradient products
+    // and waiting for P^T / dS^T no longer holds back the next S^T.
     constexpr uint32_t idesc_s = idesc_bf16(128, kQc, false, false);
-    constexpr uint32_t idesc_g = idesc_bf16(128, D, false, true);
+    const uint64_t kd0 = sdesc(smem_u32(sm.k), 16, 1024);
     bool ok = total == 0 || mbar_wait(b_kv, 0, abort_flag, status_word, 3);
-    const uint64_t kd0 = sdesc(smem_u32(sm.k), 16, 1024), vd0 = sdesc(smem_u32(sm.v), 16, 1024);
-    auto issue_s = [&](int c) -> bool {
+    for (int c = 0; ok && c < total; ++c) {
       const int st = c % kQStages;
       if (!mbar_wait(smem_u32(&sm.bar_q_full[st]), (c / kQStages) & 1, abort_flag, status_word,
-                     5))
-        return false;
-      if (c > 0 && !mbar_wait(b_xf, (c - 1) & 1, abort_flag, status_word, 6)) return false;
+                     5) ||
+          (c > 0 && !mbar_wait(b_xf, (c - 1) & 1, abort_flag, status_word, 6))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16, 1024);
 #pragma unroll
@@ -509,32 +531,42 @@ __global__ void __launch_bounds__(384, 1)
         mma_bf16(t_x, desc_at(kd0, off), desc_at(qd, off), idesc_s, k > 0 ? 1u : 0u);
       }
       mma_commit(b_s);
-      return true;
-    };
-    auto issue_dp = [&](int c) -> bool {
-      const int ds = c % kDoStages;
-      if (!mbar_wait(smem_u32(&sm.bar_do_full[ds]), (c / kDoStages) & 1, abort_flag, status_word,
-                     5))
-        return false;
-      tc_fence_after();
-      const uint64_t dd = sdesc(smem_u32(sm.dout[ds]), 16, 1024);
+    }
+  } else if (warp == 3 && lane == 0) {
+    // ------------------------------------------------------------ dP^T, dV, dK issuer
+    constexpr uint32_t idesc_s = idesc_bf16(128, kQc, false, false);
+    constexpr uint32_t idesc_g = idesc_bf16(128, D, false, true);
+    const uint64_t vd0 = sdesc(smem_u32(sm.v), 16, 1024);
+    auto issue_dp = [&](int c) {
+      const uint64_t dd = sdesc(smem_u32(sm.dout[c % kDoStages]), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
         mma_bf16(t_y, desc_at(vd0, off), desc_at(dd, off), idesc_s, k > 0 ? 1u : 0u);
       }
       mma_commit(b_dp);
-      return true;
     };
-    auto issue_grads = [&](int c) -> bool {
-      if (!mbar_wait(b_pds, c & 1, abort_flag, status_word, 4)) return false;
+    bool ok = total == 0 || (mbar_wait(b_kv, 0, abort_flag, status_word, 3) &&
+                             mbar_wait(smem_u32(&sm.bar_do_full[0]), 0, abort_flag, status_word, 5));
+    if (ok && total > 0) {
       tc_fence_after();
-      const int st = c % kQStages, ds = c % kDoStages;
+      issue_dp(0);
+    }
+    for (int c = 0; ok && c < total; ++c) {
+      const int st = c % kQStages, ds = c % kDoStages, dn = (c + 1) % kDoStages;
+      if (!mbar_wait(b_pds, c & 1, abort_flag, status_word, 4) ||
+          (c + 1 < total && !mbar_wait(smem_u32(&sm.bar_do_full[dn]), ((c + 1) / kDoStages) & 1,
+                                       abort_flag, status_word, 5))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
       // B operands MN-major: K = 16 queries per step (16 rows of 128 B), the
       // two 64-column halves of D one 16 KB box apart
       const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16384, 1024);
       const uint64_t dd = sdesc(smem_u32(sm.dout[ds]), 16384, 1024);
-      // dK += dS^T Q, then dV += P^T dO (K = 128 queries)
+      // dK += dS^T Q, then dV += P^T dO (K = 128 queries); Q(c) is released
+      // here: S^T(c) read it before the P^T threads could finish chunk c
 #pragma unroll
       for (int k = 0; k < kQc / 16; ++k)
         mma_bf16_ts(t_dk, t_y + (k >> 1) * 32 + 16 + (k & 1) * 8, desc_at(qd, k * 2048), idesc_g,
@@ -545,13 +577,7 @@ __global__ void __launch_bounds__(384, 1)
         mma_bf16_ts(t_dv, t_y + (k >> 1) * 32 + (k & 1) * 8, desc_at(dd, k * 2048), idesc_g,
                     (c > 0 || k > 0) ? 1u : 0u);
       mma_commit(smem_u32(&sm.bar_do_empty[ds]));
-      return true;
-    };
-    if (ok && total > 0) ok = issue_s(0) && issue_dp(0);
-    for (int c = 0; ok && c < total; ++c) {
-      if (c + 1 < total && !issue_s(c + 1)) ok = false;
-      else if (!issue_grads(c)) ok = false;
-      else if (c + 1 < total && !issue_dp(c + 1)) ok = false;
+      if (c + 1 < total) issue_dp(c + 1);
     }
     if (ok && total > 0) mma_commit(b_acc);
   } else if (warp >= 4) {
