@@ -15,7 +15,9 @@
 //                      into TMEM, dS by 256 threads (two per row) written back
 //                      to TMEM as bf16, dQ += dS K (A operand from TMEM)
 //                      accumulated in TMEM; K and V come through separate
-//                      rings so V is refilled as soon as dP is done.
+//                      rings so V is refilled as soon as dP is done.  S / dP
+//                      and dQ are issued by two threads, so waiting for one
+//                      stream's inputs never holds back the other's MMAs.
 //   dkdv_sm100_kernel  key-stationary (one CTA per 128-row key tile and kv
 //                      head, the plan's backward work order): over every
 //                      128-row query tile of every q head of the group that
@@ -504,25 +506,21 @@ __global__ void __launch_bounds__(384, 1)
                 status_word, 2);
     if (total > 0) mbar_wait(b_kv, 0, abort_flag, status_word, 2);
   } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------ S^T issuer
-    // Two issuing threads: this one issues S^T(c) = K Q^T into X, warp 3 the
-    // dV / dK products and dP^T(c+1) into Y (in that order: one thread's MMAs
-    // run in order, so dP^T(c+1) overwrites Y only after the gradient
-    // products have read P^T and dS^T from it).  An mbarrier wait holds the
-    // thread that executes it until the MMAs it has queued are done; split,
-    // waiting for the next Q tile no longer holds back the gradient products
-    // and waiting for P^T / dS^T no longer holds back the next S^T.
+    // ------------------------------------------------------------ MMA issuer
+    // Issue order per chunk c: S^T(c+1), dK(c), dV(c), dP^T(c+1).  S^T(c+1)
+    // overwrites X once the P^T threads hold S^T(c); dP^T(c+1) overwrites Y
+    // after dK(c) / dV(c) have read P^T and dS^T from it: tcgen05 MMAs issued
+    // by one thread run in order.
     constexpr uint32_t idesc_s = idesc_bf16(128, kQc, false, false);
-    const uint64_t kd0 = sdesc(smem_u32(sm.k), 16, 1024);
+    constexpr uint32_t idesc_g = idesc_bf16(128, D, false, true);
     bool ok = total == 0 || mbar_wait(b_kv, 0, abort_flag, status_word, 3);
-    for (int c = 0; ok && c < total; ++c) {
+    const uint64_t kd0 = sdesc(smem_u32(sm.k), 16, 1024), vd0 = sdesc(smem_u32(sm.v), 16, 1024);
+    auto issue_s = [&](int c) -> bool {
       const int st = c % kQStages;
       if (!mbar_wait(smem_u32(&sm.bar_q_full[st]), (c / kQStages) & 1, abort_flag, status_word,
-                     5) ||
-          (c > 0 && !mbar_wait(b_xf, (c - 1) & 1, abort_flag, status_word, 6))) {
-        ok = false;
-        break;
-      }
+                     5))
+        return false;
+      if (c > 0 && !mbar_wait(b_xf, (c - 1) & 1, abort_flag, status_word, 6)) return false;
       tc_fence_after();
       const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16, 1024);
 #pragma unroll
@@ -531,42 +529,32 @@ __global__ void __launch_bounds__(384, 1)
         mma_bf16(t_x, desc_at(kd0, off), desc_at(qd, off), idesc_s, k > 0 ? 1u : 0u);
       }
       mma_commit(b_s);
-    }
-  } else if (warp == 3 && lane == 0) {
-    // ------------------------------------------------------------ dP^T, dV, dK issuer
-    constexpr uint32_t idesc_s = idesc_bf16(128, kQc, false, false);
-    constexpr uint32_t idesc_g = idesc_bf16(128, D, false, true);
-    const uint64_t vd0 = sdesc(smem_u32(sm.v), 16, 1024);
-    auto issue_dp = [&](int c) {
-      const uint64_t dd = sdesc(smem_u32(sm.dout[c % kDoStages]), 16, 1024);
+      return true;
+    };
+    auto issue_dp = [&](int c) -> bool {
+      const int ds = c % kDoStages;
+      if (!mbar_wait(smem_u32(&sm.bar_do_full[ds]), (c / kDoStages) & 1, abort_flag, status_word,
+                     5))
+        return false;
+      tc_fence_after();
+      const uint64_t dd = sdesc(smem_u32(sm.dout[ds]), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
         mma_bf16(t_y, desc_at(vd0, off), desc_at(dd, off), idesc_s, k > 0 ? 1u : 0u);
       }
       mma_commit(b_dp);
+      return true;
     };
-    bool ok = total == 0 || (mbar_wait(b_kv, 0, abort_flag, status_word, 3) &&
-                             mbar_wait(smem_u32(&sm.bar_do_full[0]), 0, abort_flag, status_word, 5));
-    if (ok && total > 0) {
+    auto issue_grads = [&](int c) -> bool {
+      if (!mbar_wait(b_pds, c & 1, abort_flag, status_word, 4)) return false;
       tc_fence_after();
-      issue_dp(0);
-    }
-    for (int c = 0; ok && c < total; ++c) {
-      const int st = c % kQStages, ds = c % kDoStages, dn = (c + 1) % kDoStages;
-      if (!mbar_wait(b_pds, c & 1, abort_flag, status_word, 4) ||
-          (c + 1 < total && !mbar_wait(smem_u32(&sm.bar_do_full[dn]), ((c + 1) / kDoStages) & 1,
-                                       abort_flag, status_word, 5))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+      const int st = c % kQStages, ds = c % kDoStages;
       // B operands MN-major: K = 16 queries per step (16 rows of 128 B), the
       // two 64-column halves of D one 16 KB box apart
       const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16384, 1024);
       const uint64_t dd = sdesc(smem_u32(sm.dout[ds]), 16384, 1024);
-      // dK += dS^T Q, then dV += P^T dO (K = 128 queries); Q(c) is released
-      // here: S^T(c) read it before the P^T threads could finish chunk c
+      // dK += dS^T Q, then dV += P^T dO (K = 128 queries)
 #pragma unroll
       for (int k = 0; k < kQc / 16; ++k)
         mma_bf16_ts(t_dk, t_y + (k >> 1) * 32 + 16 + (k & 1) * 8, desc_at(qd, k * 2048), idesc_g,
@@ -577,7 +565,13 @@ __global__ void __launch_bounds__(384, 1)
         mma_bf16_ts(t_dv, t_y + (k >> 1) * 32 + (k & 1) * 8, desc_at(dd, k * 2048), idesc_g,
                     (c > 0 || k > 0) ? 1u : 0u);
       mma_commit(smem_u32(&sm.bar_do_empty[ds]));
-      if (c + 1 < total) issue_dp(c + 1);
+      return true;
+    };
+    if (ok && total > 0) ok = issue_s(0) && issue_dp(0);
+    for (int c = 0; ok && c < total; ++c) {
+      if (c + 1 < total && !issue_s(c + 1)) ok = false;
+      else if (!issue_grads(c)) ok = false;
+      else if (c + 1 < total && !issue_dp(c + 1)) ok = false;
     }
     if (ok && total > 0) mma_commit(b_acc);
   } else if (warp >= 4) {
