@@ -384,15 +384,19 @@ struct ChunkWalk {
 };
 
 // TMEM columns: dK [0, D), dV [D, 2D), X = S^T at 2D, Y = dP^T at 2D + 128
-// (128 columns each).  Two threads per key row, one per query half
-// [64 qh, 64 qh + 64): each reads its S^T half from X (freeing X for the next
-// chunk's S^T as soon as every thread has it in registers), then, 32 queries
-// at a time, reads dP^T from Y and writes P^T and dS^T (bf16 pairs, 16
-// columns each) over the 32 columns it read.  K-step k (queries 16k..16k+15)
-// of the dV product reads P^T at Y + 32 (k / 2) + 8 (k % 2), that of the dK
-// product dS^T 16 columns further.
+// (128 columns each).  Four threads per key row, one per query quarter
+// [32 qq, 32 qq + 32) (16 warps; warp w reaches TMEM lanes 32 (w % 4) ..):
+// each reads its S^T quarter from X (freeing X for the next chunk's S^T as
+// soon as every thread has it in registers), then reads dP^T from Y and
+// writes P^T and dS^T (bf16 pairs, 16 columns each) over the 32 columns it
+// read.  K-step k (queries 16k..16k+15) of the dV product reads P^T at
+// Y + 32 (k / 2) + 8 (k % 2), that of the dK product dS^T 16 columns further.
+// 576 threads: warp 0 producer, warp 1 MMA issuer, warps 2-17 P^T / dS^T.
+constexpr int kDkvThreads = 576;
+constexpr int kDkvElem = kDkvThreads - 64;   // P^T / dS^T threads
+
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kDkvThreads, 1)
     dkdv_sm100_kernel(const AttnParams a, const __grid_constant__ DkvMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -434,9 +438,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(smem_u32(&sm.bar_do_empty[s]), 1);
     }
     mbar_init(b_s, 1);
-    mbar_init(b_xf, 256);
+    mbar_init(b_xf, kDkvElem);
     mbar_init(b_dp, 1);
-    mbar_init(b_pds, 256);
+    mbar_init(b_pds, kDkvElem);
     mbar_init(b_acc, 1);
     sm.abort_flag = 0;
     mbar_fence_init();
@@ -574,11 +578,10 @@ __global__ void __launch_bounds__(384, 1)
       else if (c + 1 < total && !issue_dp(c + 1)) ok = false;
     }
     if (ok && total > 0) mma_commit(b_acc);
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ P^T, dS^T (2 threads / key)
-    const int ew = threadIdx.x - 128;
-    const int qh = ew >> 7;           // query half: [64 qh, 64 qh + 64)
-    const int row = ew & 127;
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ P^T, dS^T (4 threads / key)
+    const int qq = (warp - 2) >> 2;   // query quarter: [32 qq, 32 qq + 32)
+    const int row = (warp & 3) * 32 + lane;
     const int key = key0 + row;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
@@ -600,9 +603,8 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       tc_fence_after();
-      float p[64];
-      tmem_ld32(t_x + lane_addr + qh * 64, reinterpret_cast<uint32_t *>(p));
-      tmem_ld32(t_x + lane_addr + qh * 64 + 32, reinterpret_cast<uint32_t *>(p + 32));
+      float p[32];
+      tmem_ld32(t_x + lane_addr + qq * 32, reinterpret_cast<uint32_t *>(p));
       tc_wait_ld();
       tc_fence_before();
       mbar_arrive(b_xf);
@@ -612,39 +614,34 @@ __global__ void __launch_bounds__(384, 1)
         ok = false;
         break;
       }
-      const float4 *rec = sm.rec[ds] + qh * 64;
+      const float4 *rec = sm.rec[ds] + qq * 32;
       if (!full) {
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
+        for (int q = 0; q < 32; ++q) {
           const int2 iv =
               *reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(&rec[q]) + 8);
           if (key < iv.x || key > iv.y) p[q] = kNegInf;
         }
       }
 #pragma unroll
-      for (int q = 0; q < 64; ++q) p[q] = ex2(fmaf(p[q], sl2, -rec[q].x));
+      for (int q = 0; q < 32; ++q) p[q] = ex2(fmaf(p[q], sl2, -rec[q].x));
       if (!__all_sync(0xffffffffu, mbar_wait(b_dp, c & 1, abort_flag, status_word, 9))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      const uint32_t col = t_y + lane_addr + qq * 32;
+      float dp[32];
+      tmem_ld32(col, reinterpret_cast<uint32_t *>(dp));
+      tc_wait_ld();
+      uint32_t pk[16], dk2[16];
 #pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        const uint32_t col = t_y + lane_addr + qh * 64 + pass * 32;
-        float dp[32];
-        tmem_ld32(col, reinterpret_cast<uint32_t *>(dp));
-        tc_wait_ld();
-        uint32_t pk[16], dk2[16];
-#pragma unroll
-        for (int q = 0; q < 32; q += 2) {
-          const float p0 = p[pass * 32 + q], p1 = p[pass * 32 + q + 1];
-          pk[q / 2] = pack_bf16(p0, p1);
-          dk2[q / 2] = pack_bf16(p0 * (dp[q] - rec[pass * 32 + q].y),
-                                 p1 * (dp[q + 1] - rec[pass * 32 + q + 1].y));
-        }
-        tmem_st16(col, pk);
-        tmem_st16(col + 16, dk2);
+      for (int q = 0; q < 32; q += 2) {
+        pk[q / 2] = pack_bf16(p[q], p[q + 1]);
+        dk2[q / 2] = pack_bf16(p[q] * (dp[q] - rec[q].y), p[q + 1] * (dp[q + 1] - rec[q + 1].y));
       }
+      tmem_st16(col, pk);
+      tmem_st16(col + 16, dk2);
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(b_pds);
@@ -653,35 +650,34 @@ __global__ void __launch_bounds__(384, 1)
         !__all_sync(0xffffffffu, mbar_wait(b_acc, 0, abort_flag, status_word, 10)))
       ok = false;
     tc_fence_after();
-    // epilogue: each of the two threads of a key row stores half of dK and dV
+    // epilogue: each of the four threads of a key row stores a quarter of dK and dV
+    constexpr int kCols = D / 4;
     const bool valid = key < n_keys;
-    bf16 *dkg = (main_kv ? a.dk_m : a.dk_b) + ((int64_t)key * a.hkv + g) * D + qh * (D / 2);
-    bf16 *dvg = (main_kv ? a.dv_m : a.dv_b) + ((int64_t)key * a.hkv + g) * D + qh * (D / 2);
+    bf16 *dkg = (main_kv ? a.dk_m : a.dk_b) + ((int64_t)key * a.hkv + g) * D + qq * kCols;
+    bf16 *dvg = (main_kv ? a.dv_m : a.dv_b) + ((int64_t)key * a.hkv + g) * D + qq * kCols;
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
-      const uint32_t src = (part == 0 ? t_dk : t_dv) + qh * (D / 2);
+      const uint32_t src = (part == 0 ? t_dk : t_dv) + qq * kCols + lane_addr;
       const float mul = part == 0 ? a.scale : 1.f;
       bf16 *dst = part == 0 ? dkg : dvg;
+      uint32_t o[kCols];
+      if (ok && total > 0) {
+        if constexpr (kCols == 32) tmem_ld32(src, o);
+        else tmem_ld16(src, o);
+        tc_wait_ld();
+      } else {
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t o[32];
-        if (ok && total > 0) {
-          tmem_ld32(src + lane_addr + c * 32, o);
-          tc_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
-        if (!valid) continue;
-        uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          d4[e] = make_uint4(
-              pack_bf16(__uint_as_float(o[8 * e]) * mul, __uint_as_float(o[8 * e + 1]) * mul),
-              pack_bf16(__uint_as_float(o[8 * e + 2]) * mul, __uint_as_float(o[8 * e + 3]) * mul),
-              pack_bf16(__uint_as_float(o[8 * e + 4]) * mul, __uint_as_float(o[8 * e + 5]) * mul),
-              pack_bf16(__uint_as_float(o[8 * e + 6]) * mul, __uint_as_float(o[8 * e + 7]) * mul));
+        for (int e = 0; e < kCols; ++e) o[e] = 0u;
       }
+      if (!valid) continue;
+      uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+      for (int e = 0; e < kCols / 8; ++e)
+        d4[e] = make_uint4(
+            pack_bf16(__uint_as_float(o[8 * e]) * mul, __uint_as_float(o[8 * e + 1]) * mul),
+            pack_bf16(__uint_as_float(o[8 * e + 2]) * mul, __uint_as_float(o[8 * e + 3]) * mul),
+            pack_bf16(__uint_as_float(o[8 * e + 4]) * mul, __uint_as_float(o[8 * e + 5]) * mul),
+            pack_bf16(__uint_as_float(o[8 * e + 6]) * mul, __uint_as_float(o[8 * e + 7]) * mul));
     }
   }
 
@@ -736,13 +732,13 @@ ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s) {
   const int64_t grid_dq = (int64_t)a.n_qt * a.hq;
   const int64_t grid_kv = (int64_t)(a.n_kt + a.n_bkt) * a.hkv;
   if (d == 64) {
-    if ((st = launch_kernel(dkdv_sm100_kernel<64>, sizeof(DkvSmem<64>) + 1024, grid_kv, 384, a,
+    if ((st = launch_kernel(dkdv_sm100_kernel<64>, sizeof(DkvSmem<64>) + 1024, grid_kv, kDkvThreads, a,
                             kvm, s, "dkdv_sm100_kernel<64>")) != BA_OK)
       return st;
     return launch_kernel(dq_sm100_kernel<64>, sizeof(DqSmem<64>) + 1024, grid_dq, 384, a, dqm, s,
                          "dq_sm100_kernel<64>");
   }
-  if ((st = launch_kernel(dkdv_sm100_kernel<128>, sizeof(DkvSmem<128>) + 1024, grid_kv, 384, a,
+  if ((st = launch_kernel(dkdv_sm100_kernel<128>, sizeof(DkvSmem<128>) + 1024, grid_kv, kDkvThreads, a,
                           kvm, s, "dkdv_sm100_kernel<128>")) != BA_OK)
     return st;
   return launch_kernel(dq_sm100_kernel<128>, sizeof(DqSmem<128>) + 1024, grid_dq, 384, a, dqm, s,
