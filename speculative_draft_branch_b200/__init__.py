@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "BA_OK", -1: "BA_ERR_INVALID_ARG", -2: "BA_ERR_UNSUPPORTED",
 EXPORTS = ("ba_workspace_size", "ba_plan_layout_query", "ba_plan", "ba_plan_status",
            "branch_attn_fwd", "branch_attn_bwd", "lse_merge", "ba_set_kernel_family",
            "ba_get_kernel_family", "ba_set_kernel_events", "ba_launch_count", "ba_last_error",
-           "ba_version", "branch_attn_bwd_static_scratch", "ba_exp2_check")
+           "ba_version", "branch_attn_bwd_static_scratch", "ba_exp2_check",
+           "ba_step_host_workspace_size", "branch_attn_step_host")
 
 
 class BAProblem(ctypes.Structure):

@@ -132,6 +132,35 @@ def test_fwd_bwd_reject_misaligned_or_missing_tensors():
     assert ba.lib.branch_attn_bwd(*bargs, None) == -1
 
 
+def test_step_host_sizes_and_rejections():
+    """The host-buffer step: its staging holds every workspace and tensor, and
+    bad arguments are refused before any copy or launch."""
+    p = _problem()
+    n = ctypes.c_size_t()
+    assert ba.lib.ba_step_host_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    _, plan_b, fwd_b, bwd_b = _sizes(p)
+    d = 64
+    tensors = 2 * d * (3 * 256 * 4 + 2 * 256 * 2 + 3 * 768 * 4 + 2 * 768 * 2)  # q, o, dq / k, v
+    tensors += 2 * 2 * d * (256 * 4 + 768 * 4)                                 # dO, dK / dV extra
+    assert n.value >= plan_b + fwd_b + bwd_b + tensors
+    bad = _problem(head_dim=96)
+    assert ba.lib.ba_step_host_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == -2
+    host = [0x7000000 + i * 0x100000 for i in range(18)]
+    step = ba.lib.branch_attn_step_host
+    need = ctypes.c_size_t()
+    ba.lib.ba_step_host_workspace_size(ctypes.byref(p), ctypes.byref(need))
+    assert step(None, 0x100000, need.value, *host, None) == -1
+    assert step(ctypes.byref(p), None, need.value, *host, None) == -1
+    assert step(ctypes.byref(p), 0x100000, need.value - 1, *host, None) == -4
+    assert step(ctypes.byref(p), 0x100080, need.value, *host, None) == -3
+    missing = list(host)
+    missing[7] = None   # do_b while branch tokens exist
+    assert step(ctypes.byref(p), 0x100000, need.value, *missing, None) == -1
+    assert "null host buffer" in ba.lib.ba_last_error().decode()
+    nometa = _problem(cu_seqlens=None)
+    assert step(ctypes.byref(nometa), 0x100000, need.value, *host, None) == -1
+
+
 def test_lse_merge_rejections():
     f = ba.lib.lse_merge
     assert f(-1, 4, 64, 1, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None) == -1
