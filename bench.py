@@ -64,6 +64,18 @@ def rank_info():
             int(os.environ.get("LOCAL_RANK", 0)))
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest value over all ranks (the job's time is its slowest rank's);
+    the value itself when no process group is running."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -333,10 +345,7 @@ def run_ours(args):
     total_ms = e0.elapsed_time(e1)
     fwd_ms = [fs[i].elapsed_time(fe[i]) for i in range(K)]
     bwd_ms = [bs[i].elapsed_time(be[i]) for i in range(K)]
-    t_max = torch.tensor([total_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms = float(t_max.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_step = total_ms / K
     value = world * flops_step / (ms_step * 1e-3) / 1e12
 
@@ -402,12 +411,10 @@ def run_ours(args):
         for e, s in zip(ends, streams):
             e.record(s)
         torch.cuda.synchronize()
-        e2e_ms = torch.tensor([max(x0.elapsed_time(e) for e in ends) / E], device=dev)
-        if world > 1:
-            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * flops_step / (float(e2e_ms.item()) * 1e-3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(max(x0.elapsed_time(e) for e in ends) / E, dev)
+        e2e = {"value": world * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": float(e2e_ms.item()),
+               "ms_per_step": e2e_ms,
                "note": "branch_attn_step_host on pinned host buffers: every step uploads all "
                        "inputs and index arrays and downloads O, LSE and all six gradients; "
                        "steps alternate two streams and two staging areas"}
