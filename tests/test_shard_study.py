@@ -1,0 +1,80 @@
+"""Pins of the per-shard work count (oracle/shard_study.py) against brute
+force over the explicit mask, the total pair count, and closed forms."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+from oracle import shard_study as ss
+
+
+def _brute(st, C, order):
+    """Loop over the explicit mask: query row -> its shard, main key column ->
+    its shard; branch-key columns count on the query's own shard."""
+    dv = oracle.derive(st)
+    mask = oracle.dense_mask(st, dv)
+    n = dv.n_main
+    cu = np.asarray(dv.cu)
+    pieces = 2 * C if order == "zigzag" else C
+
+    def shard_of(pos, s):
+        start, L = int(cu[s]), int(cu[s + 1] - cu[s])
+        for k in range(pieces):
+            if start + (k * L) // pieces <= pos < start + ((k + 1) * L) // pieces:
+                return (k if k < C else 2 * C - 1 - k) if order == "zigzag" else k
+        raise AssertionError("position outside its sequence")
+
+    W = np.zeros((C, C), dtype=np.int64)
+    anchors = np.asarray(st.anchors)
+    for r in range(mask.shape[0]):
+        if r < n:
+            s, pos = int(dv.main_seq[r]), r
+        else:
+            b = int(dv.row_branch[r - n])
+            s, pos = int(dv.branch_seq[b]), int(anchors[b])
+        i = shard_of(pos, s)
+        for k in np.nonzero(mask[r, :n])[0]:
+            W[i, shard_of(int(k), int(dv.main_seq[k]))] += 1
+        W[i, i] += int(mask[r, n:].sum())
+    return W * st.hq
+
+
+@pytest.mark.parametrize("seed,kind", [(1, 0), (2, 1), (3, 2), (4, 0)])
+@pytest.mark.parametrize("C", [1, 2, 3])
+@pytest.mark.parametrize("order", ss.ORDERS)
+def test_matches_brute_force(seed, kind, C, order):
+    st = wl.random_structure(seed, n_seqs=3, max_len=30, mask_kind=kind)
+    np.testing.assert_array_equal(ss.pair_matrix(st, C, order, block=7), _brute(st, C, order))
+
+
+@pytest.mark.parametrize("order", ss.ORDERS)
+def test_total_is_the_useful_pair_count(order):
+    st = wl.structure("tiny_ttt")
+    for C in (1, 2, 4, 8):
+        assert ss.pair_matrix(st, C, order).sum() == oracle.useful_pairs(st)
+
+
+def _single_causal(L):
+    return wl.Structure("causal", np.array([0, L]), np.zeros(0, dtype=np.int64),
+                        np.zeros(0, dtype=np.int64), 1, 1, 8, 0)
+
+
+@pytest.mark.parametrize("C", [2, 4, 8])
+def test_single_causal_sequence_closed_forms(C):
+    L = 2 * C * 37
+    st = _single_causal(L)
+    zz = ss.pair_matrix(st, C, "zigzag")
+    seq = ss.pair_matrix(st, C, "sequential")
+    # zigzag: every shard does exactly L (L + 1) / (2C) pairs
+    assert np.all(zz.sum(axis=1) == L * (L + 1) // (2 * C))
+    # sequential: shard i's rows [a, b) see r + 1 keys each; no key of a later shard
+    m = L // C
+    totals = []
+    for i in range(C):
+        a, b = i * m, (i + 1) * m
+        totals.append((b * (b + 1) - a * (a + 1)) // 2)
+        assert seq[i].sum() == totals[-1]
+        assert np.all(seq[i, i + 1:] == 0)
+    assert ss.imbalance(zz)["total_max_over_mean"] == 1.0
+    assert ss.imbalance(seq)["total_max_over_mean"] == pytest.approx(
+        max(totals) / (sum(totals) / C), rel=1e-12)
