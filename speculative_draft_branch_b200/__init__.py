@@ -163,16 +163,51 @@ class Problem:
                 "lse_m": (c.hq, c.n_main), "lse_b": (c.hq, c.n_branch_tokens)}
 
 
-def _expect(t, shape, dtype, name):
+def _on_current_device(t, name):
+    """The library launches on the current CUDA device and dereferences every
+    pointer there: a host tensor or one on another device is refused here
+    instead of faulting in a kernel."""
     import torch
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (got one on {t.device})")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+
+
+def _expect(t, shape, dtype, name):
     if t is None:
         if 0 in shape:
             return
         raise ValueError(f"{name} is required")
-    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous() \
-            or (t.numel() and not t.is_cuda):
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
         raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
                          f"{t.dtype} {tuple(t.shape)} on {t.device}")
+    if t.numel():
+        _on_current_device(t, name)
+
+
+def _expect_ws(t, name):
+    """A workspace: any dtype, contiguous, on the current device."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel():
+        _on_current_device(t, name)
+
+
+def _expect_index_arrays(problem, where):
+    """ba_plan reads the index arrays on the device; the host step copies them
+    from the host itself."""
+    for name in ("cu_seqlens", "branch_anchor", "branch_depth"):
+        t = getattr(problem, name)
+        if t.numel() == 0:
+            continue
+        if where == "device":
+            _on_current_device(t, name)
+        elif t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor for branch_attn_step_host")
 
 
 def ba_workspace_size(problem: Problem):
@@ -190,11 +225,13 @@ def ba_plan_layout_query(problem: Problem) -> dict:
 
 def ba_plan(problem: Problem, plan_ws, stream=None) -> None:
     import torch
+    _expect_index_arrays(problem, "device")
     _expect(plan_ws, (plan_ws.numel(),), torch.uint8, "plan_ws")
     _check(lib.ba_plan(ctypes.byref(problem.c), _ptr(plan_ws), plan_ws.numel(), _stream(stream)))
 
 
 def ba_plan_status(plan_ws, stream=None) -> int:
+    _expect_ws(plan_ws, "plan_ws")
     word = ctypes.c_int32()
     st = lib.ba_plan_status(_ptr(plan_ws), _stream(stream), ctypes.byref(word))
     if st not in (0, -7):
@@ -205,6 +242,9 @@ def ba_plan_status(plan_ws, stream=None) -> int:
 def branch_attn_fwd(problem: Problem, plan_ws, fwd_ws, q_m, k_m, v_m, q_b, k_b, v_b, o_m, o_b,
                     lse_m, lse_b, stream=None) -> None:
     import torch
+    _expect_ws(plan_ws, "plan_ws")
+    if fwd_ws is not None:
+        _expect_ws(fwd_ws, "fwd_ws")
     sh = problem.shapes()
     for name, t in (("q_m", q_m), ("k_m", k_m), ("v_m", v_m), ("q_b", q_b), ("k_b", k_b),
                     ("v_b", v_b)):
@@ -223,6 +263,8 @@ def branch_attn_bwd(problem: Problem, plan_ws, bwd_ws, q_m, k_m, v_m, q_b, k_b, 
                     lse_m, lse_b, do_m, do_b, dq_m, dk_m, dv_m, dq_b, dk_b, dv_b,
                     stream=None) -> None:
     import torch
+    _expect_ws(plan_ws, "plan_ws")
+    _expect_ws(bwd_ws, "bwd_ws")
     sh = problem.shapes()
     pairs = (("q_m", q_m, "q_m"), ("k_m", k_m, "k_m"), ("v_m", v_m, "v_m"), ("q_b", q_b, "q_b"),
              ("k_b", k_b, "k_b"), ("v_b", v_b, "v_b"), ("o_m", o_m, "q_m"), ("o_b", o_b, "q_b"),
@@ -249,6 +291,7 @@ def branch_attn_bwd_static_scratch(problem: Problem, plan_ws, q_m, k_m, v_m, q_b
     the library (larger problems are rejected).  Calls that overlap on the GPU
     share that array and must not run concurrently."""
     import torch
+    _expect_ws(plan_ws, "plan_ws")
     sh = problem.shapes()
     pairs = (("q_m", q_m, "q_m"), ("k_m", k_m, "k_m"), ("v_m", v_m, "v_m"), ("q_b", q_b, "q_b"),
              ("k_b", k_b, "k_b"), ("v_b", v_b, "v_b"), ("o_m", o_m, "q_m"), ("o_b", o_b, "q_b"),
@@ -301,12 +344,8 @@ def branch_attn_step_host(problem: Problem, staging, q_m, k_m, v_m, q_b, k_b, v_
         _expect_host(t, sh[like], torch.bfloat16, name)
     _expect_host(lse_m, sh["lse_m"], torch.float32, "lse_m")
     _expect_host(lse_b, sh["lse_b"], torch.float32, "lse_b")
-    for name, t in (("cu_seqlens", problem.cu_seqlens), ("branch_anchor", problem.branch_anchor),
-                    ("branch_depth", problem.branch_depth)):
-        if t.is_cuda:
-            raise ValueError(f"{name} must be a host tensor for branch_attn_step_host")
-    if not staging.is_cuda:
-        raise ValueError("staging must be a device buffer")
+    _expect_index_arrays(problem, "host")
+    _expect_ws(staging, "staging")
     nbytes = staging.numel() * staging.element_size()
     _check(lib.branch_attn_step_host(
         ctypes.byref(problem.c), _ptr(staging), nbytes, _ptr(q_m), _ptr(k_m), _ptr(v_m),
@@ -319,7 +358,7 @@ def lse_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, stream=None) -> None:
     """o_* [rows, heads, d] fp32 or bf16; lse_* [heads, rows] fp32; in place allowed."""
     import torch
     rows, heads, d = o_a.shape
-    for name, t in (("o_b", o_b), ("o_out", o_out)):
+    for name, t in (("o_a", o_a), ("o_b", o_b), ("o_out", o_out)):
         _expect(t, o_a.shape, o_a.dtype, name)
     for name, t in (("lse_a", lse_a), ("lse_b", lse_b), ("lse_out", lse_out)):
         _expect(t, (heads, rows), torch.float32, name)

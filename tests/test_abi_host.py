@@ -183,3 +183,41 @@ def test_kernel_family_switch():
             ba.ba_set_kernel_family(3)
     finally:
         ba.ba_set_kernel_family(old)
+
+
+def test_binding_refuses_host_memory_where_the_library_reads_the_device():
+    """Host tensors passed where the library dereferences device memory (the
+    index arrays at plan time, the workspaces, the operands) are refused by the
+    binding before any library call, and the host step refuses a host staging
+    buffer."""
+    import torch
+    import workloads as wl
+    st = wl.structure("tiny_ttt")
+    prob = ba.Problem.from_structure(st, device="cpu")
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="cu_seqlens must be a CUDA tensor"):
+        ba.ba_plan(prob, ws)
+    with pytest.raises(ValueError, match="plan_ws must be a CUDA tensor"):
+        ba.ba_plan_status(ws)
+    t = wl.tensors(st, 1, "cpu")
+    sh = prob.shapes()
+    o_m, o_b = torch.empty_like(t["q_m"]), torch.empty_like(t["q_b"])
+    lse_m = torch.empty(sh["lse_m"], dtype=torch.float32)
+    lse_b = torch.empty(sh["lse_b"], dtype=torch.float32)
+    fwd_in = (t["q_m"], t["k_m"], t["v_m"], t["q_b"], t["k_b"], t["v_b"])
+    with pytest.raises(ValueError, match="plan_ws must be a CUDA tensor"):
+        ba.branch_attn_fwd(prob, ws, None, *fwd_in, o_m, o_b, lse_m, lse_b)
+    grads = [torch.empty_like(t[k]) for k in ("q_m", "k_m", "v_m", "q_b", "k_b", "v_b")]
+    with pytest.raises(ValueError, match="plan_ws must be a CUDA tensor"):
+        ba.branch_attn_bwd(prob, ws, ws, *fwd_in, o_m, o_b, lse_m, lse_b, t["do_m"], t["do_b"],
+                           *grads)
+    with pytest.raises(ValueError, match="plan_ws must be a CUDA tensor"):
+        ba.branch_attn_bwd_static_scratch(prob, ws, *fwd_in, o_m, o_b, lse_m, lse_b, t["do_m"],
+                                          t["do_b"], *grads)
+    with pytest.raises(ValueError, match="staging must be a CUDA tensor"):
+        ba.branch_attn_step_host(prob, ws, *fwd_in, t["do_m"], t["do_b"], o_m, o_b, lse_m,
+                                 lse_b, *grads)
+    oa = torch.zeros(8, 2, 64)
+    la = torch.zeros(2, 8)
+    with pytest.raises(ValueError, match="o_a must be a CUDA tensor"):
+        ba.lse_merge(oa, la, oa.clone(), la.clone(), oa.clone(), la.clone())
