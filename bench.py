@@ -17,7 +17,9 @@ pairs) / step time.
 With N > 1 (torchrun) each rank runs an independent replica of the batch
 (weak scaling: the path has no cross-GPU exchange at this layout); the step
 time is the max over ranks.  `--impl reference` times the fp64 CPU oracle on a
-bounded sample of the same workload on the host cores.
+bounded sample of the same workload on the host cores.  `--shard-timing C`
+(with a one-sequence workload) runs the tile-order study instead: per-shard
+times of the zigzag and the sequential order of C shards, from prefix timings.
 """
 from __future__ import annotations
 
@@ -56,6 +58,9 @@ def parse_args():
                     help="profile-sized case: only the first N main tokens and their branches")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shard-timing", type=int, default=0, metavar="C",
+                    help="tile-order study: per-shard fwd+bwd time of the zigzag and the "
+                         "sequential order of C shards over one sequence (prints its own line)")
     return ap.parse_args()
 
 
@@ -459,8 +464,108 @@ def run_ours(args):
     return 0
 
 
+def shard_split(prefix, C: int):
+    """Per-shard sums of an additive quantity of one sequence cut into 2C equal
+    chunks, from its values on the prefixes ending at the chunk boundaries
+    (prefix[k] covers chunks 0..k-1, prefix[0] = 0): zigzag shard i holds
+    chunks i and 2C-1-i, sequential shard i chunks 2i and 2i+1."""
+    P = 2 * C
+    if len(prefix) != P + 1:
+        raise ValueError(f"need {P + 1} prefix values, got {len(prefix)}")
+    chunk = [prefix[k + 1] - prefix[k] for k in range(P)]
+    return {"chunk": chunk,
+            "zigzag": [chunk[i] + chunk[P - 1 - i] for i in range(C)],
+            "sequential": [chunk[2 * i] + chunk[2 * i + 1] for i in range(C)]}
+
+
+def run_shard_timing(args):
+    """Timing half of the tile-order study, on one GPU.
+
+    One causal sequence (the workload cut to --tokens main tokens and their
+    branches) is split into 2C equal chunks.  The rows of a chunk [a, b) see
+    only keys below b, so their fwd+bwd time is T(b) - T(a), where T(x) is the
+    step time of the x-token prefix; timing the 2C prefixes that end at the
+    chunk boundaries gives every chunk's time and so every shard's, for the
+    zigzag and the sequential order.  Useful pairs come from the library's plan
+    of each prefix.  Each prefix: --warmup untimed steps, the median of --steps
+    timed ones (CUDA events on the launching stream)."""
+    import dataclasses
+
+    import torch
+
+    import speculative_draft_branch_b200 as ba
+    import workloads as wl
+
+    rank, _, local_rank = rank_info()
+    if rank != 0:
+        return 0
+    C = args.shard_timing
+    st_full = wl.structure(args.workload)
+    if len(st_full.cu_seqlens) != 2:
+        raise SystemExit("--shard-timing needs a one-sequence workload (ttt_256k, dspark_64k)")
+    L = args.tokens or st_full.n_main
+    P = 2 * C
+    if C < 1 or L % (P * 128) != 0 or L > st_full.n_main:
+        raise SystemExit(f"--tokens {L} must be a multiple of 2C x 128 = {P * 128} "
+                         f"and at most {st_full.n_main}")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    base = dataclasses.replace(wl.truncate(st_full, L), zigzag_C=1)
+    t_full = wl.tensors(base, wl.workload_seed(args.workload), dev)
+    stream = torch.cuda.current_stream()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    T, pairs = [0.0], [0]
+    for k in range(1, P + 1):
+        st = dataclasses.replace(wl.truncate(base, k * L // P), zigzag_C=1)
+        t = wl.slice_tensors(base, st, t_full)
+        runner = ba.BranchAttention(ba.Problem.from_structure(st, device=dev), device=dev)
+        runner.plan()
+        if runner.plan_status() != 0:
+            raise RuntimeError("plan content checks failed")
+        pairs.append(useful_pairs_from_plan(runner))
+        out, grads = runner.alloc_outputs(), runner.alloc_grads()
+        ms = []
+        for i in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            runner.forward(t, out)
+            runner.backward(t, out, grads)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ms.append(e0.elapsed_time(e1))
+        if runner.plan_status() != 0:
+            raise RuntimeError("a device-side check failed during the timed steps")
+        T.append(statistics.median(ms))
+        del runner, out, grads, t
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    tm, pr = shard_split(T, C), shard_split(pairs, C)
+    d = base.head_dim
+
+    def ratio(x):
+        return max(x) / (sum(x) / len(x))
+
+    print(json.dumps({
+        "study": "shard_timing", "workload": args.workload, "tokens": L, "C": C,
+        "steps": args.steps, "warmup": args.warmup, "prefix_ms": T[1:],
+        "chunk_ms": tm["chunk"], "chunk_pairs": pr["chunk"],
+        "chunk_tflops": [10 * d * p / (m * 1e-3) / 1e12 if m > 0 else None
+                         for p, m in zip(pr["chunk"], tm["chunk"])],
+        "zigzag": {"shard_ms": tm["zigzag"], "max_over_mean_time": ratio(tm["zigzag"]),
+                   "max_over_mean_pairs": ratio(pr["zigzag"])},
+        "sequential": {"shard_ms": tm["sequential"],
+                       "max_over_mean_time": ratio(tm["sequential"]),
+                       "max_over_mean_pairs": ratio(pr["sequential"])},
+        "clocks": clk}))
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.shard_timing:
+        return run_shard_timing(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -78,3 +78,25 @@ def test_single_causal_sequence_closed_forms(C):
     assert ss.imbalance(zz)["total_max_over_mean"] == 1.0
     assert ss.imbalance(seq)["total_max_over_mean"] == pytest.approx(
         max(totals) / (sum(totals) / C), rel=1e-12)
+
+
+@pytest.mark.parametrize("C", [2, 4])
+def test_prefix_differences_give_the_shard_totals(C):
+    """bench.py's shard timing turns totals over the 2C prefixes of one sequence
+    into per-shard sums; fed each prefix's useful-pair count it must give the
+    pair matrix's shard totals, for both orders (the decomposition behind the
+    measured per-shard times)."""
+    import dataclasses
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    L = 2 * C * 48
+    base = dataclasses.replace(wl.truncate(wl.structure("ttt_256k"), L), zigzag_C=1)
+    prefix = [0] + [oracle.useful_pairs(wl.truncate(base, k * L // (2 * C)))
+                    for k in range(1, 2 * C + 1)]
+    split = bench.shard_split(prefix, C)
+    for order in ss.ORDERS:
+        np.testing.assert_array_equal(split[order], ss.pair_matrix(base, C, order).sum(axis=1))
+    with pytest.raises(ValueError):
+        bench.shard_split(prefix[:-1], C)
