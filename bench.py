@@ -149,13 +149,20 @@ class ClockSampler:
                 "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
 
 
+# The sources that decide what the profiled launches do: the tcgen05 kernels
+# and their headers, the backward preprocess, the plan (work order) and the
+# dispatch.  Host staging (step_host.cu), the static-scratch entry and the
+# mma.sync family do not change those launches.
+PROFILED_SOURCES = ("api.cu", "attn_sm100.cu", "attn_sm100_bwd.cu", "attn_sm100_common.cuh",
+                    "internal.cuh", "merge.cu", "plan.cu", "sm100.cuh")
+
+
 def kernel_source_sha():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "speculative_draft_branch_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+    for f in PROFILED_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 

@@ -27,17 +27,29 @@ struct CopyStreams {
 std::mutex g_mu;
 CopyStreams g_streams[kMaxDevices];
 
+void destroy(CopyStreams &c) {
+  for (cudaStream_t s : {c.up, c.down})
+    if (s) cudaStreamDestroy(s);
+  for (cudaEvent_t ev : {c.start, c.in_fwd, c.in_bwd, c.fwd, c.bwd, c.done})
+    if (ev) cudaEventDestroy(ev);
+}
+
+// Created all at once on first use per device: a partly created set is
+// destroyed and never published, so a later call retries from scratch.
 ba_status copy_streams(int dev, CopyStreams **out) {
   CopyStreams &c = g_streams[dev];
   if (!c.up) {
-    cudaError_t e;
-    if ((e = cudaStreamCreateWithFlags(&c.up, cudaStreamNonBlocking)) != cudaSuccess ||
-        (e = cudaStreamCreateWithFlags(&c.down, cudaStreamNonBlocking)) != cudaSuccess)
-      return cuda_check(e, "creating the copy streams");
-    cudaEvent_t *evs[6] = {&c.start, &c.in_fwd, &c.in_bwd, &c.fwd, &c.bwd, &c.done};
+    CopyStreams n;
+    cudaError_t e = cudaStreamCreateWithFlags(&n.up, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&n.down, cudaStreamNonBlocking);
+    cudaEvent_t *evs[6] = {&n.start, &n.in_fwd, &n.in_bwd, &n.fwd, &n.bwd, &n.done};
     for (cudaEvent_t *ev : evs)
-      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
-        return cuda_check(e, "creating the copy events");
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      destroy(n);
+      return cuda_check(e, "creating the copy streams and events");
+    }
+    c = n;
   }
   *out = &c;
   return BA_OK;
