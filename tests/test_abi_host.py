@@ -221,3 +221,31 @@ def test_binding_refuses_host_memory_where_the_library_reads_the_device():
     la = torch.zeros(2, 8)
     with pytest.raises(ValueError, match="o_a must be a CUDA tensor"):
         ba.lse_merge(oa, la, oa.clone(), la.clone(), oa.clone(), la.clone())
+
+
+def test_package_fails_loudly_without_the_library(tmp_path):
+    """The binding without libbranch_attn.so does not import: there is no
+    fallback path to take instead."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "speculative_draft_branch_b200"
+    pkg.mkdir()
+    src = os.path.join(ROOT, "speculative_draft_branch_b200")
+    for f in ("__init__.py", "runner.py"):
+        shutil.copy(os.path.join(src, f), pkg / f)
+    r = subprocess.run([sys.executable, "-c", "import speculative_draft_branch_b200"],
+                       cwd=tmp_path, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "build.py" in r.stderr
+
+
+def test_product_sources_do_not_reach_the_oracle():
+    """Neither the package nor the C interface imports, links or names the
+    CPU oracle: it is test infrastructure only."""
+    for base in (os.path.join(ROOT, "speculative_draft_branch_b200"), os.path.join(ROOT, "include")):
+        for dirpath, _, files in os.walk(base):
+            for f in files:
+                if f.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
+                    text = open(os.path.join(dirpath, f)).read()
+                    assert not re.search(r"\boracle\b", text, flags=re.I), os.path.join(dirpath, f)
