@@ -269,6 +269,19 @@ BA_API ba_status lse_merge(int64_t rows, int32_t heads, int32_t head_dim,
 BA_API ba_status ba_exp2_check(const float *x, float *y_fma, float *y_hw, int64_t n,
                                ba_stream_t stream);
 
+/* Device self-check of failure detection (no counterpart in the paper).  One
+ * thread waits, with the bounded mbarrier wait every tcgen05 kernel uses
+ * (limit 2 s), on an mbarrier in shared memory.  arrive = 1: the thread
+ * arrives on it first and the wait completes at once.  arrive = 0: nothing
+ * arrives, the wait gives up after its limit and sets bit 15 of the plan
+ * workspace's device-timeout word, as a kernel whose wait gave up does, so
+ * ba_plan_status then returns BA_ERR_DEVICE_TIMEOUT (ba_plan clears it).
+ * Nothing traps or faults; the context stays usable.  plan_ws: a workspace
+ * written by ba_plan (device pointer, 16-byte aligned); async on `stream`.
+ * Returns BA_ERR_INVALID_ARG for a NULL workspace or another arrive value,
+ * BA_ERR_MISALIGNED for a misaligned one. */
+BA_API ba_status ba_wait_check(void *plan_ws, int32_t arrive, ba_stream_t stream);
+
 /* Kernel family for the attention kernels:
  *   0 = default (tcgen05/TMEM/TMA kernels),
  *   1 = tcgen05/TMEM/TMA kernels,

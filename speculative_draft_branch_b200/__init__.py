@@ -32,7 +32,7 @@ EXPORTS = ("ba_workspace_size", "ba_plan_layout_query", "ba_plan", "ba_plan_stat
            "branch_attn_fwd", "branch_attn_bwd", "lse_merge", "ba_set_kernel_family",
            "ba_get_kernel_family", "ba_set_kernel_events", "ba_launch_count", "ba_last_error",
            "ba_version", "branch_attn_bwd_static_scratch", "ba_exp2_check",
-           "ba_step_host_workspace_size", "branch_attn_step_host")
+           "ba_step_host_workspace_size", "branch_attn_step_host", "ba_wait_check")
 
 
 class BAProblem(ctypes.Structure):
@@ -80,6 +80,7 @@ def _load() -> ctypes.CDLL:
         "ba_get_kernel_family": [],
         "ba_set_kernel_events": [I32, VP, VP],
         "ba_exp2_check": [VP, VP, VP, I64, VP],
+        "ba_wait_check": [VP, I32, VP],
         "ba_step_host_workspace_size": [P, ctypes.POINTER(S)],
         "branch_attn_step_host": [P, VP, S] + [VP] * 18 + [VP],
         "ba_launch_count": [],
@@ -390,6 +391,15 @@ def ba_exp2_check(x, stream=None):
     y_fma, y_hw = torch.empty_like(x), torch.empty_like(x)
     _check(lib.ba_exp2_check(_ptr(x), _ptr(y_fma), _ptr(y_hw), x.numel(), _stream(stream)))
     return y_fma, y_hw
+
+
+def ba_wait_check(plan_ws, arrive: bool, stream=None) -> None:
+    """Failure-detection self-check: a bounded device wait on a barrier that is
+    (arrive=True) or is not (arrive=False) arrived on; in the second case the
+    wait gives up after 2 s and ba_plan_status(plan_ws) then reports
+    BA_ERR_DEVICE_TIMEOUT.  Asynchronous on `stream`."""
+    _expect_ws(plan_ws, "plan_ws")
+    _check(lib.ba_wait_check(_ptr(plan_ws), 1 if arrive else 0, _stream(stream)))
 
 
 def ba_launch_count() -> int:

@@ -223,19 +223,22 @@ def test_binding_refuses_host_memory_where_the_library_reads_the_device():
         ba.lse_merge(oa, la, oa.clone(), la.clone(), oa.clone(), la.clone())
 
 
-def test_package_fails_loudly_without_the_library(tmp_path):
+def test_package_fails_loudly_without_the_library():
     """The binding without libbranch_attn.so does not import: there is no
     fallback path to take instead."""
     import shutil
     import subprocess
     import sys
-    pkg = tmp_path / "speculative_draft_branch_b200"
-    pkg.mkdir()
-    src = os.path.join(ROOT, "speculative_draft_branch_b200")
-    for f in ("__init__.py", "runner.py"):
-        shutil.copy(os.path.join(src, f), pkg / f)
-    r = subprocess.run([sys.executable, "-c", "import speculative_draft_branch_b200"],
-                       cwd=tmp_path, capture_output=True, text=True, timeout=300)
+    import tempfile
+    os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+    with tempfile.TemporaryDirectory(dir=os.path.join(ROOT, "_build")) as tmp:
+        pkg = os.path.join(tmp, "speculative_draft_branch_b200")
+        os.mkdir(pkg)
+        src = os.path.join(ROOT, "speculative_draft_branch_b200")
+        for f in ("__init__.py", "runner.py"):
+            shutil.copy(os.path.join(src, f), os.path.join(pkg, f))
+        r = subprocess.run([sys.executable, "-c", "import speculative_draft_branch_b200"],
+                           cwd=tmp, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert "ImportError" in r.stderr and "build.py" in r.stderr
 
@@ -249,3 +252,13 @@ def test_product_sources_do_not_reach_the_oracle():
                 if f.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
                     text = open(os.path.join(dirpath, f)).read()
                     assert not re.search(r"\boracle\b", text, flags=re.I), os.path.join(dirpath, f)
+
+
+def test_wait_check_rejections():
+    """The failure-detection self-check refuses a missing or misaligned plan
+    workspace and an unknown mode before launching."""
+    f = ba.lib.ba_wait_check
+    assert f(None, 0, None) == -1
+    assert f(0x100008, 0, None) == -3
+    assert f(0x100000, 2, None) == -1
+    assert "arrive" in ba.lib.ba_last_error().decode()
