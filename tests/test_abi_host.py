@@ -262,3 +262,41 @@ def test_wait_check_rejections():
     assert f(0x100008, 0, None) == -3
     assert f(0x100000, 2, None) == -1
     assert "arrive" in ba.lib.ba_last_error().decode()
+
+
+def test_struct_layouts_match_the_header():
+    """The binding's ctypes mirrors of ba_problem and ba_plan_layout have the
+    header's size and field offsets, as the host C compiler lays them out."""
+    import shutil
+    import subprocess
+    import tempfile
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    mirrors = {"ba_problem": ba.BAProblem, "ba_plan_layout": ba.BAPlanLayout}
+    src = ["#include <stdio.h>", "#include <stddef.h>", '#include "branch_attn.h"',
+           "int main(void) {"]
+    for name, cls in mirrors.items():
+        src.append(f'  printf("{name} sizeof %zu\\n", sizeof({name}));')
+        for field, _ in cls._fields_:
+            src.append(f'  printf("{name} {field} %zu\\n", offsetof({name}, {field}));')
+    src += ["  return 0;", "}"]
+    os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+    with tempfile.TemporaryDirectory(dir=os.path.join(ROOT, "_build")) as tmp:
+        c_file, exe = os.path.join(tmp, "layout.c"), os.path.join(tmp, "layout")
+        with open(c_file, "w") as f:
+            f.write("\n".join(src) + "\n")
+        subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        c_file, "-o", exe], check=True, timeout=120)
+        out = subprocess.run([exe], check=True, capture_output=True, text=True,
+                             timeout=60).stdout
+    seen = 0
+    for line in out.splitlines():
+        name, field, value = line.split()
+        cls = mirrors[name]
+        if field == "sizeof":
+            assert ctypes.sizeof(cls) == int(value), name
+        else:
+            assert getattr(cls, field).offset == int(value), (name, field)
+        seen += 1
+    assert seen == sum(len(c._fields_) + 1 for c in mirrors.values())
