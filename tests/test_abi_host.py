@@ -300,3 +300,18 @@ def test_struct_layouts_match_the_header():
             assert getattr(cls, field).offset == int(value), (name, field)
         seen += 1
     assert seen == sum(len(c._fields_) + 1 for c in mirrors.values())
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every entry point's ctypes argtypes has as many entries as the header
+    declares parameters."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    decls = re.findall(r"BA_API\s+[\w\s\*]+?\b(\w+)\s*\(([^)]*)\)\s*;", text, flags=re.S)
+    assert decls
+    for name, params in decls:
+        params = params.strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        fn = getattr(ba.lib, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
