@@ -286,6 +286,78 @@ def run_reference(args):
     return 0
 
 
+# ---------------------------------------------------------------- HBM-bound steps
+def hbm_steps(ba, runner, t, out, grads, stream, dev, hbm_gbs, max_rows=1 << 18):
+    """Achieved GB/s of the path's two HBM-bound steps against the measured
+    copy bandwidth, timed after the step loop.
+
+    lse_merge: fp32 partials for every row and head of the workload (at most
+    max_rows rows), several GB, so each call reads more than L2 holds; CUDA
+    events around 10 calls after 3 warm-up calls.  Per (row, head) it reads
+    2 d fp32 values and 2 LSE values and writes d values and 1 LSE value.
+
+    D preprocess: launched inside branch_attn_bwd ahead of the attention
+    kernels, so its time is the backward call's span minus the span of the
+    attention kernels (both CUDA events on the launching stream); that
+    difference also holds two launch gaps.  Per (row, head) it reads O and dO
+    (2 d bf16) and the LSE and writes D and two 16-byte records; per row it
+    reads the 16-byte key interval."""
+    import torch
+    c = runner.problem.c
+    rows, heads, d = c.n_main + c.n_branch_tokens, c.hq, c.head_dim
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def roof(nbytes, ms, **extra):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return dict(achieved=gbs, peak=hbm_gbs, unit="GB/s", frac=gbs / hbm_gbs,
+                    bytes_per_launch=int(nbytes), ms=ms, **extra)
+
+    res = {}
+    m_rows = min(rows, max_rows)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    o_a = torch.randn((m_rows, heads, d), generator=gen, device=dev)
+    o_b = torch.randn((m_rows, heads, d), generator=gen, device=dev)
+    l_a = torch.randn((heads, m_rows), generator=gen, device=dev)
+    l_b = torch.randn((heads, m_rows), generator=gen, device=dev)
+    o_o, l_o = torch.empty_like(o_a), torch.empty_like(l_a)
+    for _ in range(3):
+        ba.lse_merge(o_a, l_a, o_b, l_b, o_o, l_o)
+    e0, e1 = ev(), ev()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(10):
+        ba.lse_merge(o_a, l_a, o_b, l_b, o_o, l_o)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    res["lse_merge"] = roof(m_rows * heads * (3 * d * 4 + 3 * 4), e0.elapsed_time(e1) / 10,
+                            rows=m_rows, partials="fp32")
+    del o_a, o_b, l_a, l_b, o_o, l_o
+
+    ks, ke, c0, c1 = ev(), ev(), ev(), ev()
+    for e in (ks, ke):      # torch creates the event handle on first record
+        e.record(stream)
+    torch.cuda.synchronize()
+    spans = []
+    try:
+        for i in range(5):
+            ba.ba_set_kernel_events(1, ks, ke)
+            c0.record(stream)
+            runner.backward(t, out, grads)
+            c1.record(stream)
+            torch.cuda.synchronize()
+            if i >= 2:
+                spans.append(c0.elapsed_time(c1) - ks.elapsed_time(ke))
+    finally:
+        ba.ba_set_kernel_events(1, None, None)
+    res["bwd_preprocess"] = roof(rows * heads * (2 * d * 2 + 4 + 4 + 32) + rows * 16,
+                                 statistics.median(spans),
+                                 note="time = backward call span minus attention-kernel span")
+    return res
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -450,6 +522,14 @@ def run_ours(args):
                     "extrapolated_note": "EXTRAPOLATED: the workload's useful pairs over the "
                                          "sampled fp64 pairs per second"}
 
+    hbm = None
+    if rank == 0:
+        try:
+            hbm = hbm_steps(ba, runner, t, out, grads, stream, dev,
+                            float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])))
+        except Exception as exc:  # reported in the line; never costs the headline
+            hbm = {"error": repr(exc)[:300]}
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -469,6 +549,7 @@ def run_ours(args):
                                         "the step loop)",
                          "algorithmic": f"{'10' if dom == 'bwd' else '4'} d x {pairs} pairs "
                                         "per launch"},
+            "hbm_steps": hbm,
             "cpu_baseline": cpu_base,
             "e2e": e2e,
             "gpu_launches": int(launches),

@@ -1,0 +1,75 @@
+"""Host logic of bench.py's HBM-step measurement, run on the CPU with fake
+CUDA events and a fake library, so every line executes and the byte
+accounting is checked against hand-computed figures."""
+import os
+import sys
+import types
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+class _Clock:
+    t = 0.0
+
+
+class _FakeEvent:
+    """Records a tick of a shared clock; elapsed_time is the tick difference (ms)."""
+
+    def __init__(self, enable_timing=True):
+        self.stamp = None
+        self.cuda_event = 1
+
+    def record(self, stream=None):
+        _Clock.t += 1.0
+        self.stamp = _Clock.t
+
+    def elapsed_time(self, other):
+        return other.stamp - self.stamp
+
+
+def test_hbm_steps_byte_accounting(monkeypatch):
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setattr(torch.cuda, "Event", _FakeEvent)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    calls = {"merge": 0, "bwd": 0, "events": []}
+    ks_ke = {}
+
+    def lse_merge(o_a, l_a, o_b, l_b, o_o, l_o, stream=None):
+        assert o_a.shape == o_b.shape == o_o.shape and l_a.shape == (o_a.shape[1], o_a.shape[0])
+        calls["merge"] += 1
+
+    def set_events(which, start=None, stop=None):
+        assert which == 1
+        calls["events"].append(start is not None)
+        ks_ke["pair"] = (start, stop)
+
+    ba = types.SimpleNamespace(lse_merge=lse_merge, ba_set_kernel_events=set_events)
+
+    class Runner:
+        problem = types.SimpleNamespace(c=types.SimpleNamespace(
+            n_main=1000, n_branch_tokens=3000, hq=4, head_dim=64))
+
+        def backward(self, t, out, grads):
+            # the library records its kernel events around the attention kernels
+            calls["bwd"] += 1
+            start, stop = ks_ke["pair"]
+            start.record()
+            stop.record()
+
+    res = bench.hbm_steps(ba, Runner(), {}, {}, {}, None, "cpu", hbm_gbs=1000.0, max_rows=2500)
+    assert calls["merge"] == 13 and calls["bwd"] == 5
+    assert calls["events"][-1] is False           # events switched off afterwards
+    m = res["lse_merge"]
+    assert m["rows"] == 2500                      # capped at max_rows
+    assert m["bytes_per_launch"] == 2500 * 4 * (3 * 64 * 4 + 3 * 4)
+    assert m["ms"] == pytest.approx(0.1)          # 10 calls between two ticks
+    p = res["bwd_preprocess"]
+    # call span c0 -> c1 is 3 ticks (kernel start, kernel stop, end), kernel span 1 tick
+    assert p["ms"] == pytest.approx(2.0)
+    assert p["bytes_per_launch"] == 4000 * 4 * (2 * 64 * 2 + 4 + 4 + 32) + 4000 * 16
+    assert p["frac"] == pytest.approx(p["achieved"] / 1000.0)
+    assert p["achieved"] == pytest.approx(p["bytes_per_launch"] / 2e-3 / 1e9)
