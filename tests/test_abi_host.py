@@ -315,3 +315,25 @@ def test_binding_argument_counts_match_the_header():
         fn = getattr(ba.lib, name)
         assert fn.argtypes is not None, name
         assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
+def test_plain_c_caller_links_and_runs():
+    """A C program (tests/c/host_caller.c) compiles against the header, links
+    the shared library and gets the documented results from the calls that
+    need no GPU."""
+    import shutil
+    import subprocess
+    import tempfile
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    lib_dir = os.path.dirname(ba.LIB_PATH)
+    os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+    with tempfile.TemporaryDirectory(dir=os.path.join(ROOT, "_build")) as tmp:
+        exe = os.path.join(tmp, "host_caller")
+        subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c", "host_caller.c"), "-o", exe,
+                        "-L", lib_dir, "-lbranch_attn", f"-Wl,-rpath,{lib_dir}"],
+                       check=True, timeout=120)
+        r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
