@@ -100,21 +100,26 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.out = None
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        scratch = os.path.join(ROOT, "_build")
+        os.makedirs(scratch, exist_ok=True)
+        fd, self.path = tempfile.mkstemp(suffix=".csv", dir=scratch)
+        self.out = os.fdopen(fd, "w")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                stdout=self.out, stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.proc = None
         time.sleep(0.3)
 
     def stop(self):
         if self.proc is None:
+            self.out.close()
+            os.unlink(self.path)
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.25)
         self.proc.terminate()
@@ -122,6 +127,8 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
+            self.proc.wait(timeout=5)
+        self.out.close()
         rows = []
         with open(self.path) as f:
             for line in f:

@@ -73,3 +73,47 @@ def test_hbm_steps_byte_accounting(monkeypatch):
     assert p["bytes_per_launch"] == 4000 * 4 * (2 * 64 * 2 + 4 + 4 + 32) + 4000 * 16
     assert p["frac"] == pytest.approx(p["achieved"] / 1000.0)
     assert p["achieved"] == pytest.approx(p["bytes_per_launch"] / 2e-3 / 1e9)
+
+
+def test_clock_sampler_parses_samples_and_reasons(monkeypatch):
+    """ClockSampler against a stand-in nvidia-smi printing three samples: the
+    median SM clock is taken over the samples under load, throttle reasons are
+    the ones reported Active, and the sampler cleans up after itself."""
+    import stat
+    import tempfile
+    sys.path.insert(0, ROOT)
+    import bench
+    lines = ["0, 1500, 1965, 900.5, 0x4, Not Active, Not Active, Not Active, Active",
+             "0, 300, 1965, 100.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+             "0, 1520, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active"]
+    os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+    with tempfile.TemporaryDirectory(dir=os.path.join(ROOT, "_build")) as tmp:
+        fake = os.path.join(tmp, "nvidia-smi")
+        with open(fake, "w") as f:
+            f.write("#!/usr/bin/env python3\nimport time\n")
+            for ln in lines:
+                f.write(f"print({ln!r}, flush=True)\n")
+            f.write("time.sleep(60)\n")
+        os.chmod(fake, os.stat(fake).st_mode | stat.S_IXUSR)
+        monkeypatch.setenv("PATH", tmp + os.pathsep + os.environ["PATH"])
+        cs = bench.ClockSampler(0)
+        cs.start()
+        import time
+        time.sleep(1.0)
+        clk = cs.stop()
+        assert not os.path.exists(cs.path) and cs.out.closed
+    assert clk["samples"] == 3
+    assert clk["sm_mhz"] == pytest.approx(1510.0)
+    assert clk["sm_max_mhz"] == pytest.approx(1965.0)
+    assert clk["reasons"] == ["sw_power_cap"]
+    assert clk["power_w_max"] == pytest.approx(950.0)
+
+
+def test_clock_sampler_without_nvidia_smi(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("PATH", os.path.join(ROOT, "no-such-dir"))
+    cs = bench.ClockSampler(0)
+    cs.start()
+    clk = cs.stop()
+    assert clk["reasons"] == ["nvidia-smi unavailable"] and not os.path.exists(cs.path)
