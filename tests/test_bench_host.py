@@ -117,3 +117,23 @@ def test_clock_sampler_without_nvidia_smi(monkeypatch):
     cs.start()
     clk = cs.stop()
     assert clk["reasons"] == ["nvidia-smi unavailable"] and not os.path.exists(cs.path)
+
+
+def test_profiled_traffic_only_for_the_profiled_sources(monkeypatch):
+    """The traffic figure of a profile summary is used only while its source
+    hash matches the current kernel sources."""
+    import tempfile
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "00c0ffee00c0ffee")
+    os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+    with tempfile.TemporaryDirectory(dir=os.path.join(ROOT, "_build")) as tmp:
+        os.mkdir(os.path.join(tmp, "profiles"))
+        monkeypatch.setattr(bench, "ROOT", tmp)
+        with open(os.path.join(tmp, "profiles", "bwd_attention_w.md"), "w") as f:
+            f.write("traffic_bytes_per_launch: 2.5e9\nsource_sha: 00c0ffee00c0ffee\n")
+        with open(os.path.join(tmp, "profiles", "fwd_attention_w.md"), "w") as f:
+            f.write("traffic_bytes_per_launch: 1.0e9\nsource_sha: 1111111111111111\n")
+        assert bench.profiled_traffic("bwd_attention", "w") == 2.5e9
+        assert bench.profiled_traffic("fwd_attention", "w") is None     # stale profile
+        assert bench.profiled_traffic("bwd_attention", "other") is None  # no profile
