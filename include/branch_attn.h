@@ -151,7 +151,9 @@ typedef struct {
  * fwd_bytes:  scratch of branch_attn_fwd (0 when zigzag_C == 1; otherwise
  *   fp32 accumulators of O and LSE for every query row and head).
  * bwd_bytes:  scratch of branch_attn_bwd: D = rowsum(dO * O) fp32
- *   [Hq, rows] and the fp32 dQ accumulator [rows, Hq, d]. */
+ *   [Hq, rows], per-query records {LSE log2 e, D, first key, last key}
+ *   (float4, twice per row and head, rows padded to 128 per token kind) and
+ *   the fp32 dQ accumulator [rows, Hq, d] of the fused backward. */
 BA_API ba_status ba_workspace_size(const ba_problem *p, size_t *plan_bytes,
                             size_t *fwd_bytes, size_t *bwd_bytes);
 
@@ -206,14 +208,17 @@ BA_API ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws,
  * reserves its whole HBM budget in its own pool at start-up, or a plugin whose
  * host forbids allocation at run time) and cannot cudaMalloc the backward
  * workspace.  This call takes the same arguments as branch_attn_bwd minus the
- * workspace and keeps its scratch (D plus the fp32 dQ accumulator or the
- * per-query backward records) in a 32 MiB array compiled into the library,
+ * workspace and keeps its scratch (D, the per-query backward records and the
+ * fp32 dQ accumulator) in a 32 MiB array compiled into the library,
  * which every GPU that loads the library holds until exit.  It allocates
  * nothing.
  *   - Problems whose backward scratch (see ba_workspace_size) exceeds 32 MiB
  *     are rejected with BA_ERR_WORKSPACE_TOO_SMALL before any launch.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is looked up again when the device's context changes (after
+ *     cudaDeviceReset, for example): an address from a context that no longer
+ *     exists is never reused.
  *   - All calls on a device share the array; each call re-initialises what it
  *     needs, but calls whose kernels overlap on the GPU race on it. */
 BA_API ba_status branch_attn_bwd_static_scratch(
@@ -239,7 +244,9 @@ BA_API ba_status branch_attn_bwd_static_scratch(
  *   - Host buffers should be page-locked; pageable memory works but the
  *     copies then do not overlap.
  *   - The host outputs are complete once `stream` reaches the point after
- *     this call.  Inputs must stay unchanged until then.
+ *     this call.  Inputs must stay unchanged until then.  A call that returns
+ *     an error has waited for every copy it had already queued, so its host
+ *     buffers are free again when it returns.
  *   - Plan content errors are not checked here; ba_plan_status on the plan
  *     inside the staging area (at offset 0) reports them after the step. */
 BA_API ba_status ba_step_host_workspace_size(const ba_problem *p, size_t *bytes);
@@ -282,21 +289,27 @@ BA_API ba_status ba_exp2_check(const float *x, float *y_fma, float *y_hw, int64_
  * BA_ERR_MISALIGNED for a misaligned one. */
 BA_API ba_status ba_wait_check(void *plan_ws, int32_t arrive, ba_stream_t stream);
 
-/* Kernel family for the attention kernels:
- *   0 = default (tcgen05/TMEM/TMA kernels),
- *   1 = tcgen05/TMEM/TMA kernels,
- *   2 = warp-level mma.sync kernels (the pre-Blackwell tensor-core path, kept
- *       as a second independent implementation).
+/* Backward kernel family (the forward is the same for both):
+ *   0 = default: one fused tcgen05 kernel per (key tile, kv head) computing
+ *       S, dP, dV, dK and dQ (the method's five tile products); dQ partials
+ *       are summed in fp32 in the workspace and converted to bf16 by a final
+ *       pass, so dQ may differ in the last bits from run to run (the order of
+ *       the fp32 sums is not fixed); dK and dV are deterministic;
+ *   1 = split backward: a key-stationary dK/dV kernel and a query-stationary
+ *       dQ kernel (S and dP computed twice, seven tile products), every
+ *       gradient written once in bf16; bit-reproducible from run to run.
  * Returns BA_ERR_INVALID_ARG for other values.  Process-wide. */
 BA_API ba_status ba_set_kernel_family(int32_t family);
 BA_API int32_t ba_get_kernel_family(void);
 
 /* Benchmark instrumentation.  After ba_set_kernel_events(which, start, stop)
  * every later call records the caller-owned CUDA event `start` (a cudaEvent_t)
- * on the call's stream right before its attention kernel and `stop` right
- * after it (which = 0: branch_attn_fwd, 1: branch_attn_bwd; for the zigzag
- * forward the pair brackets all ring-step launches).  NULL events switch it
- * off.  Process-wide; not for concurrent use from several threads. */
+ * on the call's stream right before its attention kernels and `stop` right
+ * after them (which = 0: branch_attn_fwd, all ring-step launches of the
+ * zigzag forward included; 1: branch_attn_bwd's attention kernels and the dQ
+ * conversion, without the preprocess; 2: branch_attn_bwd's preprocess
+ * kernel D = rowsum(dO * O) alone).  NULL events switch it off.
+ * Process-wide; not for concurrent use from several threads. */
 BA_API ba_status ba_set_kernel_events(int32_t which, void *start_event, void *stop_event);
 
 /* Number of kernel launches the library has issued in this process. */

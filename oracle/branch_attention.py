@@ -15,7 +15,7 @@ Shapes of the three draft-branch kinds (TTT-causal, block-bidirectional,
 block-causal) follow the EAGLE-3 / DFlash / DSpark description in the
 research-background section.
 
-Conventions (the reading stated in the design notes):
+Conventions (readings of the pages where they leave a point open):
   * main tokens t = 0..N-1 packed by cu_seqlens; branch b has anchor a_b and
     depth D_b, its tokens are branch rows cu_branch[b] .. cu_branch[b+1]-1
     (anchor-major, depth-minor);
@@ -308,6 +308,29 @@ def _row_sets(st, dv, main_rows, branch_rows):
     return items
 
 
+# Rows of one sequence are scored together in batches of at most this many
+# score-matrix entries (rows x main keys), so that full-size sequences fit in
+# host memory; batching changes which rows share a matmul, not any value.
+ROW_BATCH_ENTRIES = 1 << 24
+
+
+def _row_batches(items, idx):
+    """Split the row indices `idx` of one sequence into batches of rows with
+    similar main-key counts, each batch's score matrix within ROW_BATCH_ENTRIES."""
+    order = sorted(idx, key=lambda i: items[i][2].size)
+    batches, cur, width = [], [], 0
+    for i in order:
+        w = max(width, items[i][2].size)
+        if cur and w * (len(cur) + 1) > ROW_BATCH_ENTRIES:
+            batches.append(cur)
+            cur, w = [], items[i][2].size
+        cur.append(i)
+        width = w
+    if cur:
+        batches.append(cur)
+    return batches
+
+
 def rows_forward(st, t, main_rows=(), branch_rows=(), with_dq=False, heads=None):
     """Forward (and optionally dQ) of selected query rows, each over its own key set.
 
@@ -316,8 +339,9 @@ def rows_forward(st, t, main_rows=(), branch_rows=(), with_dq=False, heads=None)
     all) are computed; the others stay zero.
 
     Rows reading the same sequence share one score matrix S = K_prefix q^T
-    (a plain matmul); each row then masks the keys it does not see (main keys
-    past its own position / anchor) and appends its branch-local scores.
+    (a plain matmul, taken over batches of rows); each row then masks the keys
+    it does not see (main keys past its own position / anchor) and appends its
+    branch-local scores.
     """
     dv = derive(st)
     items = _row_sets(st, dv, main_rows, branch_rows)
@@ -332,7 +356,8 @@ def rows_forward(st, t, main_rows=(), branch_rows=(), with_dq=False, heads=None)
     for i, (kind, r, mk, lk) in enumerate(items):
         by_seq.setdefault(int(dv.main_seq[mk[0]]), []).append(i)
     groups = sorted({h // grp for h in heads})
-    for s, idx in by_seq.items():
+    batches = [(s, b) for s, idx in by_seq.items() for b in _row_batches(items, idx)]
+    for s, idx in batches:
         lo = int(dv.cu[s])
         hi = max(int(items[i][2][-1]) for i in idx) + 1
         nm = np.array([items[i][2].size for i in idx])            # main keys per row
@@ -414,6 +439,21 @@ def keys_backward(st, t, main_keys=(), branch_keys=(), groups=None):
     q_branch = sorted(q_branch)
     fw = rows_forward(st, t, q_main, q_branch, heads=heads)
     items = _row_sets(st, dv, q_main, q_branch)
+    R = len(items)
+    # visibility of every selected key from every visiting row: main keys in
+    # the row's main interval, branch keys in its branch-local interval
+    m_lo = np.array([it[2][0] for it in items], dtype=np.int64)
+    m_hi = np.array([it[2][-1] for it in items], dtype=np.int64)
+    b_lo = np.array([it[3][0] if it[3].size else 0 for it in items], dtype=np.int64)
+    b_hi = np.array([it[3][-1] if it[3].size else -1 for it in items], dtype=np.int64)
+    vis_m = (main_keys[None, :] >= m_lo[:, None]) & (main_keys[None, :] <= m_hi[:, None])
+    vis_b = (branch_keys[None, :] >= b_lo[:, None]) & (branch_keys[None, :] <= b_hi[:, None])
+    qx = np.zeros((R, hq, d))
+    dox = np.zeros((R, hq, d))
+    for i, (kind, r, _, _) in enumerate(items):
+        sfx = "m" if kind == "main" else "b"
+        qx[i] = to64(t["q_" + sfx][r])
+        dox[i] = to64(t["do_" + sfx][r])
     km_sel = to64(t["k_m"][main_keys]) if main_keys.size else np.zeros((0, hkv, d))
     vm_sel = to64(t["v_m"][main_keys]) if main_keys.size else np.zeros((0, hkv, d))
     kb_sel = to64(t["k_b"][branch_keys]) if branch_keys.size else np.zeros((0, hkv, d))
@@ -422,26 +462,18 @@ def keys_backward(st, t, main_keys=(), branch_keys=(), groups=None):
     dv_m = np.zeros((main_keys.size, hkv, d))
     dk_b = np.zeros((branch_keys.size, hkv, d))
     dv_b = np.zeros((branch_keys.size, hkv, d))
-    for i, (kind, r, mk, lk) in enumerate(items):
-        sel_m = np.nonzero((main_keys >= mk[0]) & (main_keys <= mk[-1]))[0]
-        sel_b = (np.nonzero((branch_keys >= lk[0]) & (branch_keys <= lk[-1]))[0]
-                 if lk.size else np.zeros(0, dtype=np.int64))
-        if sel_m.size == 0 and sel_b.size == 0:
-            continue
-        sfx = "m" if kind == "main" else "b"
-        qx = to64(t["q_" + sfx][r])
-        dox = to64(t["do_" + sfx][r])
-        for h in heads:
-            g = h // grp
-            dd = float(dox[h] @ fw["o"][i, h])
-            for sel, ksel, vsel, dk, dvv in ((sel_m, km_sel, vm_sel, dk_m, dv_m),
-                                            (sel_b, kb_sel, vb_sel, dk_b, dv_b)):
-                if sel.size == 0:
-                    continue
-                p = np.exp(st.scale * (ksel[sel, g] @ qx[h]) - fw["lse"][h, i])
-                ds = p * (vsel[sel, g] @ dox[h] - dd)
-                dvv[sel, g] += p[:, None] * dox[h][None]
-                dk[sel, g] += st.scale * ds[:, None] * qx[h][None]
+    for h in heads:
+        g = h // grp
+        dd = (dox[:, h] * fw["o"][:, h]).sum(axis=1)                # D_i = dO_i . O_i
+        for vis, ksel, vsel, dk, dvv in ((vis_m, km_sel, vm_sel, dk_m, dv_m),
+                                         (vis_b, kb_sel, vb_sel, dk_b, dv_b)):
+            if ksel.shape[0] == 0:
+                continue
+            s_ik = st.scale * (qx[:, h] @ ksel[:, g].T)             # [R, keys]
+            p = np.where(vis, np.exp(np.where(vis, s_ik, 0.0) - fw["lse"][h][:, None]), 0.0)
+            ds = p * (dox[:, h] @ vsel[:, g].T - dd[:, None])
+            dvv[:, g] += p.T @ dox[:, h]
+            dk[:, g] += st.scale * (ds.T @ qx[:, h])
     return {"dk_m": dk_m, "dv_m": dv_m, "dk_b": dk_b, "dv_b": dv_b}
 
 
@@ -463,3 +495,69 @@ def useful_pairs(st) -> int:
         loc = depth * (depth + 1) // 2
     branch = int((pre * depth + loc).sum())
     return (main + branch) * st.hq
+
+
+def visible_counts(st, dv: Derived = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Number of keys each main row and each branch row sees (mask definition):
+    main row r of sequence s sees r - cu[s] + 1 keys; branch token j of branch
+    b (anchor a, depth D) sees a - cu[s] + 1 main keys plus j + 1 (causal
+    kinds) or D (block-bidirectional) keys of its branch."""
+    dv = dv or derive(st)
+    n_m = np.arange(dv.n_main) - dv.cu[dv.main_seq] + 1
+    anchors = np.asarray(st.anchors, dtype=np.int64)
+    b = dv.row_branch
+    j = np.arange(dv.n_branch_tokens) - dv.cu_branch[b]
+    depth = dv.cu_branch[b + 1] - dv.cu_branch[b]
+    pre = anchors[b] - dv.cu[dv.branch_seq[b]] + 1 if b.size else np.zeros(0, dtype=np.int64)
+    loc = depth if st.mask_kind == MASK_BLOCK_BIDIR else j + 1
+    return n_m.astype(np.int64), (pre + loc).astype(np.int64)
+
+
+def zero_query_dv(st, t, groups=None):
+    """dV of every main and branch key when every query is zero.
+
+    With q = 0 every visible score is 0, so P_ik = 1 / n_i over the n_i keys
+    row i sees (visible_counts), and the backward definition gives
+    dV_k = sum over the rows i that see key k of dO_i / n_i (summed over the q
+    heads of k's kv group) and dK_k = scale sum_i dS_ik q_i = 0.
+      * main key k of sequence s is seen by the main rows i >= k of s and by
+        every token of the branches of s anchored at a position >= k, so its
+        dV is a suffix sum over the positions of s of w_i = dO_i / n_i plus,
+        at each anchor position, the branch tokens' w;
+      * branch key (b, j') is seen by the tokens (b, j) with j >= j' (causal
+        kinds: a suffix sum within the branch) or by every token of b
+        (block-bidirectional: the branch total).
+    Only kv heads in `groups` (default all) are filled; returns dv_m [N, Hkv, d]
+    and dv_b [Nb, Hkv, d] in fp64.
+    """
+    dv = derive(st)
+    hq, hkv, d = st.hq, st.hkv, st.head_dim
+    grp = hq // hkv
+    groups = list(range(hkv)) if groups is None else [int(g) for g in groups]
+    n_m, n_b = visible_counts(st, dv)
+    n, nb = dv.n_main, dv.n_branch_tokens
+    anchors = np.asarray(st.anchors, dtype=np.int64)
+    seq_end = dv.cu[dv.main_seq + 1]                  # end of each main token's sequence
+    out_m = np.zeros((n, hkv, d))
+    out_b = np.zeros((nb, hkv, d))
+    for g in groups:
+        for h in range(g * grp, (g + 1) * grp):
+            w_m = to64(t["do_m"][:, h]) / n_m[:, None]
+            w_b = to64(t["do_b"][:, h]) / n_b[:, None] if nb else np.zeros((0, d))
+            tot = w_m.copy()
+            if nb:
+                per_branch = np.zeros((anchors.size, d))
+                np.add.at(per_branch, dv.row_branch, w_b)
+                np.add.at(tot, anchors, per_branch)
+            # G[k] = sum_{i >= k} tot_i; the suffix within k's sequence is G[k] - G[end]
+            G = np.zeros((n + 1, d))
+            G[:n] = np.cumsum(tot[::-1], axis=0)[::-1]
+            out_m[:, g] += G[:n] - G[seq_end]
+            if nb:
+                if st.mask_kind == MASK_BLOCK_BIDIR:
+                    out_b[:, g] += per_branch[dv.row_branch]
+                else:
+                    Gb = np.zeros((nb + 1, d))
+                    Gb[:nb] = np.cumsum(w_b[::-1], axis=0)[::-1]
+                    out_b[:, g] += Gb[:nb] - Gb[dv.cu_branch[dv.row_branch + 1]]
+    return out_m, out_b

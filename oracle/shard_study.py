@@ -82,7 +82,7 @@ def imbalance(W: np.ndarray) -> Dict[str, float]:
             "ring_time_over_ideal": float(sum(x.max() for x in steps) / (totals.sum() / C))}
 
 
-if __name__ == "__main__":  # the table quoted in the design notes
+if __name__ == "__main__":  # prints the imbalance table of the three batches
     import workloads as wl
     for name in ("ttt_20k", "dflash_32k", "ttt_256k"):
         st = wl.structure(name)

@@ -3,12 +3,14 @@
     python speculative_draft_branch_b200/build.py [--force] [--verbose]
 
 Every .cu file under csrc/ is compiled separately (parallel) and linked into
-one shared library next to this file.  Rebuilds only what changed.
+one shared library next to this file.  Rebuilds only what changed, judged
+by a content hash of each output's sources, headers and command line.
 """
 from __future__ import annotations
 
 import argparse
 import concurrent.futures as cf
+import hashlib
 import os
 import shutil
 import subprocess
@@ -35,15 +37,35 @@ def nvcc() -> str:
 
 def _deps() -> list:
     out = [os.path.join(INCLUDE, "branch_attn.h")]
-    out += [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
+    out += sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
     return out
 
 
-def _stale(target: str, sources: list) -> bool:
-    if not os.path.exists(target):
-        return True
-    t = os.path.getmtime(target)
-    return any(os.path.getmtime(s) > t for s in sources)
+def _digest(paths, cmd) -> str:
+    """Content hash of the files an output depends on and of the command that
+    makes it: an output is rebuilt whenever this changes, whatever the files'
+    modification times say (a checkout or a copy can leave a built library
+    newer than sources it was not built from)."""
+    h = hashlib.sha256()
+    h.update("\0".join(cmd).encode())
+    for p in paths:
+        h.update(p.encode())
+        with open(p, "rb") as f:
+            h.update(hashlib.sha256(f.read()).digest())
+    return h.hexdigest()
+
+
+def _fresh(target: str, digest: str) -> bool:
+    stamp = target + ".sha256"
+    if not (os.path.exists(target) and os.path.exists(stamp)):
+        return False
+    with open(stamp) as f:
+        return f.read().strip() == digest
+
+
+def _stamp(target: str, digest: str) -> None:
+    with open(target + ".sha256", "w") as f:
+        f.write(digest + "\n")
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
@@ -56,28 +78,33 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         src = os.path.join(CSRC, f)
         obj = os.path.join(OBJ, f[:-3] + ".o")
         objs.append(obj)
-        if force or _stale(obj, [src] + deps):
-            cmd = [nvcc()] + ARCH + FLAGS + list(extra) + ["-c", src, "-o", obj]
+        cmd = [nvcc()] + ARCH + FLAGS + list(extra) + ["-c", src, "-o", obj]
+        digest = _digest([src] + deps, cmd[1:])
+        if force or not _fresh(obj, digest):
             if verbose:
                 cmd.insert(1, "-Xptxas=-v")
-            jobs.append(cmd)
+            jobs.append((cmd, obj, digest))
 
-    def run(cmd):
+    def run(job):
+        cmd, obj, digest = job
         r = subprocess.run(cmd, capture_output=True, text=True)
-        return cmd, r
+        return job, r
 
     with cf.ThreadPoolExecutor(max_workers=min(8, max(1, len(jobs)))) as ex:
-        for cmd, r in ex.map(run, jobs):
+        for (cmd, obj, digest), r in ex.map(run, jobs):
             if verbose or r.returncode != 0:
                 sys.stderr.write(r.stdout + r.stderr)
             if r.returncode != 0:
                 raise RuntimeError("nvcc failed: " + " ".join(cmd))
-    if force or jobs or _stale(LIB, objs):
-        cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs
-        r = subprocess.run(cmd, capture_output=True, text=True)
+            _stamp(obj, digest)
+    link = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs
+    lib_digest = _digest(objs, link[1:])
+    if force or jobs or not _fresh(LIB, lib_digest):
+        r = subprocess.run(link, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError("link failed")
+        _stamp(LIB, lib_digest)
     return LIB
 
 

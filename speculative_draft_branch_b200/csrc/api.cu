@@ -14,8 +14,8 @@ namespace {
 thread_local char g_err[1024] = "";
 std::atomic<int> g_family{0};
 std::atomic<int64_t> g_launches{0};
-std::atomic<void *> g_ev_start[2] = {nullptr, nullptr};
-std::atomic<void *> g_ev_stop[2] = {nullptr, nullptr};
+std::atomic<void *> g_ev_start[3] = {nullptr, nullptr, nullptr};
+std::atomic<void *> g_ev_stop[3] = {nullptr, nullptr, nullptr};
 
 void record_event(int which, bool start, cudaStream_t s) {
   void *ev = start ? g_ev_start[which].load() : g_ev_stop[which].load();
@@ -161,13 +161,17 @@ size_t rows_padded(const ba_problem &p) {
   return align_up((size_t)p.n_main, 128) + align_up((size_t)p.n_branch_tokens, 128);
 }
 
-// D [Hq, rows] fp32, then one region used either as the fp32 dQ accumulator
-// (mma.sync backward) or as the per-query records (tcgen05 backward).
+// Backward workspace, three regions at 256-byte offsets:
+//   D        [Hq, rows] fp32, rowsum(dO * O)
+//   records  [2][Hq][rows padded to 128 per kind] float4 {LSE log2 e, D, key lo, key hi}
+//   dQ acc   [rows, Hq, d] fp32 (the fused backward's dQ accumulator)
+size_t bwd_d_bytes(const ba_problem &p) {
+  return align_up(4 * ((size_t)p.n_main + p.n_branch_tokens) * p.hq, 256);
+}
+size_t bwd_rec_bytes(const ba_problem &p) { return align_up(2 * 16 * rows_padded(p) * p.hq, 256); }
 size_t bwd_ws_bytes(const ba_problem &p) {
   const size_t rows = (size_t)p.n_main + p.n_branch_tokens;
-  const size_t acc = 4 * rows * p.hq * p.head_dim;
-  const size_t rec = 2 * 16 * rows_padded(p) * p.hq;
-  return align_up(4 * rows * p.hq, 256) + align_up(acc > rec ? acc : rec, 256);
+  return bwd_d_bytes(p) + bwd_rec_bytes(p) + align_up(4 * rows * p.hq * p.head_dim, 256);
 }
 
 AttnParams make_params(const ba_problem &p, const ba_plan_layout &L, const void *plan_ws) {
@@ -213,8 +217,6 @@ ba_status check_plan_ws(const void *plan_ws) {
   return BA_OK;
 }
 
-bool use_sm100_fwd() { return g_family.load() != 2 && sm100_fwd_available(); }
-bool use_sm100_bwd() { return g_family.load() != 2 && sm100_bwd_available(); }
 
 #define BA_TRY(expr)                   \
   do {                                 \
@@ -312,10 +314,7 @@ ba_status branch_attn_fwd(const ba_problem *p, const void *plan_ws, void *fwd_ws
   a.o_m = (__nv_bfloat16 *)o_m; a.o_b = (__nv_bfloat16 *)o_b;
   a.lse_m = lse_m; a.lse_b = lse_b;
   cudaStream_t s = (cudaStream_t)stream;
-  const bool sm100 = use_sm100_fwd();
-  auto launch = [&](const AttnParams &x) {
-    return sm100 ? launch_fwd_sm100(x, s) : launch_fwd_mma(x, s);
-  };
+  auto launch = [&](const AttnParams &x) { return launch_fwd_sm100(x, s); };
   if (p->zigzag_C <= 1) {
     record_event(0, true, s);
     ba_status st = launch(a);
@@ -371,28 +370,28 @@ ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws, void *bwd_ws
   a.do_m = (const __nv_bfloat16 *)do_m; a.do_b = (const __nv_bfloat16 *)do_b;
   a.dk_m = (__nv_bfloat16 *)dk_m; a.dv_m = (__nv_bfloat16 *)dv_m;
   a.dk_b = (__nv_bfloat16 *)dk_b; a.dv_b = (__nv_bfloat16 *)dv_b;
-  const size_t rows = (size_t)p->n_main + p->n_branch_tokens;
-  a.d_all = reinterpret_cast<const float *>(bwd_ws);
-  a.dq_acc = reinterpret_cast<float *>(reinterpret_cast<char *>(bwd_ws) +
-                                       align_up(4 * rows * p->hq, 256));
-  cudaStream_t s = (cudaStream_t)stream;
+  char *ws = reinterpret_cast<char *>(bwd_ws);
+  a.d_all = reinterpret_cast<const float *>(ws);
+  a.rec = reinterpret_cast<float4 *>(ws + bwd_d_bytes(*p));
+  a.dq_acc = reinterpret_cast<float *>(ws + bwd_d_bytes(*p) + bwd_rec_bytes(*p));
+  a.n_main_pad = (int32_t)align_up((size_t)p->n_main, 128);
+  a.rows_pad = (int32_t)rows_padded(*p);
   a.dq_out_m = (__nv_bfloat16 *)dq_m;
   a.dq_out_b = (__nv_bfloat16 *)dq_b;
-  const bool sm100 = use_sm100_bwd();
-  // tcgen05: dK/dV and dQ kernels write every gradient directly;
-  // mma.sync: dQ is accumulated in fp32 with atomics, then converted
-  a.zero_dq_acc = sm100 ? 0 : 1;
-  if (sm100) {
-    a.rec = reinterpret_cast<float4 *>(a.dq_acc);
-    a.n_main_pad = (int32_t)align_up((size_t)p->n_main, 128);
-    a.rows_pad = (int32_t)rows_padded(*p);
-  }
+  cudaStream_t s = (cudaStream_t)stream;
+  // family 0: one fused kernel accumulating dQ in fp32 (the preprocess zeroes
+  // the accumulator, a last pass converts it); family 1: the deterministic
+  // split backward (dK/dV kernel + dQ kernel, both writing bf16 directly)
+  const bool fused = g_family.load() == 0 && sm100_fused_bwd_available();
+  a.zero_dq_acc = fused ? 1 : 0;
+  record_event(2, true, s);
   BA_TRY(launch_bwd_preprocess(a, s));
+  record_event(2, false, s);
   record_event(1, true, s);
-  BA_TRY(sm100 ? launch_bwd_sm100(a, s) : launch_bwd_mma(a, s));
+  BA_TRY(fused ? launch_bwd_fused_sm100(a, s) : launch_bwd_sm100(a, s));
+  if (fused) BA_TRY(launch_dq_convert(a, (__nv_bfloat16 *)dq_m, (__nv_bfloat16 *)dq_b, s));
   record_event(1, false, s);
-  if (sm100) return BA_OK;
-  return launch_dq_convert(a, (__nv_bfloat16 *)dq_m, (__nv_bfloat16 *)dq_b, s);
+  return BA_OK;
 }
 
 ba_status lse_merge(int64_t rows, int32_t heads, int32_t head_dim, int32_t o_is_fp32,
@@ -431,7 +430,7 @@ ba_status ba_exp2_check(const float *x, float *y_fma, float *y_hw, int64_t n, ba
 }
 
 ba_status ba_set_kernel_family(int32_t family) {
-  if (family < 0 || family > 2) {
+  if (family < 0 || family > 1) {
     set_error("unknown kernel family %d", family);
     return BA_ERR_INVALID_ARG;
   }
@@ -442,8 +441,8 @@ ba_status ba_set_kernel_family(int32_t family) {
 int32_t ba_get_kernel_family(void) { return g_family.load(); }
 
 ba_status ba_set_kernel_events(int32_t which, void *start_event, void *stop_event) {
-  if (which < 0 || which > 1) {
-    set_error("ba_set_kernel_events: which must be 0 (forward) or 1 (backward)");
+  if (which < 0 || which > 2) {
+    set_error("ba_set_kernel_events: which must be 0 (forward), 1 (backward) or 2 (preprocess)");
     return BA_ERR_INVALID_ARG;
   }
   g_ev_start[which].store(start_event);

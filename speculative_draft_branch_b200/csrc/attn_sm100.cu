@@ -85,6 +85,7 @@ struct FwdSmem {
   uint64_t bar_p_full[2];
   uint64_t bar_o_done;
   uint64_t bar_o_final;  // one phase: the last PV product has landed in O
+  uint64_t bar_drain;    // one phase: every MMA the issuer queued has completed
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     mbar_init(b_o, 1);
     mbar_init(b_final, 1);
+    mbar_init(smem_u32(&sm.bar_drain), 1);
     sm.abort_flag = 0;
     mbar_fence_init();
   }
@@ -185,12 +187,10 @@ __global__ void __launch_bounds__(256, 1)
     }
     // on abort: let the loads already issued land before the CTA exits
     for (int j = (issued_k > kFwdStages ? issued_k - kFwdStages : 0); j < issued_k; ++j)
-      mbar_wait(smem_u32(&sm.bar_k_full[j % kFwdStages]), (j / kFwdStages) & 1, abort_flag,
-                status_word, 2);
+      mbar_wait_drain(smem_u32(&sm.bar_k_full[j % kFwdStages]), (j / kFwdStages) & 1, status_word, 2);
     for (int j = (issued_v > kFwdStages ? issued_v - kFwdStages : 0); j < issued_v; ++j)
-      mbar_wait(smem_u32(&sm.bar_v_full[j % kFwdStages]), (j / kFwdStages) & 1, abort_flag,
-                status_word, 2);
-    if (total > 0) mbar_wait(b_q, 0, abort_flag, status_word, 2);
+      mbar_wait_drain(smem_u32(&sm.bar_v_full[j % kFwdStages]), (j / kFwdStages) & 1, status_word, 2);
+    if (total > 0) mbar_wait_drain(b_q, 0, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
@@ -238,6 +238,9 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
     if (ok && total > 0 && issue_pv(total - 1)) mma_commit(b_final);
+    // nothing may still write TMEM when it is freed, aborted or not
+    mma_commit(smem_u32(&sm.bar_drain));
+    mbar_wait_drain(smem_u32(&sm.bar_drain), 0, status_word, 2);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
     const int row = threadIdx.x - 128;
@@ -462,6 +465,7 @@ struct Fwd2Smem {
   uint64_t bar_v_full[kFwd2Stages], bar_v_empty[kFwd2Stages];
   uint64_t bar_s_full[2], bar_p_full[2];
   uint64_t bar_o_final;
+  uint64_t bar_drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -504,6 +508,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(smem_u32(&sm.bar_p_full[x]), 128);
     }
     mbar_init(b_final, 1);
+    mbar_init(smem_u32(&sm.bar_drain), 1);
     sm.abort_flag = 0;
     mbar_fence_init();
   }
@@ -562,12 +567,10 @@ __global__ void __launch_bounds__(384, 1)
       ++issued_v;
     }
     for (int j = (issued_k > kFwd2Stages ? issued_k - kFwd2Stages : 0); j < issued_k; ++j)
-      mbar_wait(smem_u32(&sm.bar_k_full[j % kFwd2Stages]), (j / kFwd2Stages) & 1, abort_flag,
-                status_word, 2);
+      mbar_wait_drain(smem_u32(&sm.bar_k_full[j % kFwd2Stages]), (j / kFwd2Stages) & 1, status_word, 2);
     for (int j = (issued_v > kFwd2Stages ? issued_v - kFwd2Stages : 0); j < issued_v; ++j)
-      mbar_wait(smem_u32(&sm.bar_v_full[j % kFwd2Stages]), (j / kFwd2Stages) & 1, abort_flag,
-                status_word, 2);
-    if (total > 0) mbar_wait(b_q, 0, abort_flag, status_word, 2);
+      mbar_wait_drain(smem_u32(&sm.bar_v_full[j % kFwd2Stages]), (j / kFwd2Stages) & 1, status_word, 2);
+    if (total > 0) mbar_wait_drain(b_q, 0, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
@@ -612,6 +615,8 @@ __global__ void __launch_bounds__(384, 1)
            (j + 1 >= total || issue_s(1, j + 1));
     }
     if (ok && total > 0) mma_commit(b_final);
+    mma_commit(smem_u32(&sm.bar_drain));
+    mbar_wait_drain(smem_u32(&sm.bar_drain), 0, status_word, 2);
   }
   } else {
     regs_inc<208>();
@@ -822,8 +827,6 @@ ba_status launch_exp2_check(const float *x, float *y_fma, float *y_mufu, int64_t
   return cuda_check(cudaGetLastError(), "exp2_check_kernel launch");
 }
 
-bool sm100_fwd_available() { return true; }
-bool sm100_available() { return true; }
 
 ba_status launch_fwd_sm100(const AttnParams &a, cudaStream_t s) {
   TensorMaps tm;

@@ -55,6 +55,7 @@ struct DqSmem {
   uint64_t bar_ds_full[2];  // one per dS buffer: the dS threads may run a tile ahead
   uint64_t bar_dq_done[2];  // dQ(i) has read dS buffer i % 2
   uint64_t bar_dq_final;
+  uint64_t bar_drain[2];    // per issuing thread: its queued MMAs have completed
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -109,6 +110,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(smem_u32(&sm.bar_dq_done[0]), 1);
     mbar_init(smem_u32(&sm.bar_dq_done[1]), 1);
     mbar_init(b_final, 1);
+    mbar_init(smem_u32(&sm.bar_drain[0]), 1);
+    mbar_init(smem_u32(&sm.bar_drain[1]), 1);
     sm.abort_flag = 0;
     mbar_fence_init();
   }
@@ -163,12 +166,10 @@ __global__ void __launch_bounds__(384, 1)
       ++issued_v;
     }
     for (int j = (issued_k > kDqKStages ? issued_k - kDqKStages : 0); j < issued_k; ++j)
-      mbar_wait(smem_u32(&sm.bar_k_full[j % kDqKStages]), (j / kDqKStages) & 1, abort_flag,
-                status_word, 2);
+      mbar_wait_drain(smem_u32(&sm.bar_k_full[j % kDqKStages]), (j / kDqKStages) & 1, status_word, 2);
     for (int j = (issued_v > kDqVStages ? issued_v - kDqVStages : 0); j < issued_v; ++j)
-      mbar_wait(smem_u32(&sm.bar_v_full[j % kDqVStages]), (j / kDqVStages) & 1, abort_flag,
-                status_word, 2);
-    if (total > 0) mbar_wait(b_qdo, 0, abort_flag, status_word, 2);
+      mbar_wait_drain(smem_u32(&sm.bar_v_full[j % kDqVStages]), (j / kDqVStages) & 1, status_word, 2);
+    if (total > 0) mbar_wait_drain(b_qdo, 0, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ S / dP issuer
     // Two issuing threads: this one issues S and dP of each key tile, warp 3
@@ -206,6 +207,8 @@ __global__ void __launch_bounds__(384, 1)
       mma_commit(b_sdp_full);
       mma_commit(smem_u32(&sm.bar_v_empty[vs]));
     }
+    mma_commit(smem_u32(&sm.bar_drain[0]));
+    mbar_wait_drain(smem_u32(&sm.bar_drain[0]), 0, status_word, 2);
   } else if (warp == 3 && lane == 0) {
     // ------------------------------------------------------------ dQ issuer
     // dQ(i) += dS(i) K(i).  K(i) is released here: S(i) read it before the
@@ -227,6 +230,8 @@ __global__ void __launch_bounds__(384, 1)
       mma_commit(smem_u32(&sm.bar_dq_done[i & 1]));
     }
     if (ok && total > 0) mma_commit(b_final);
+    mma_commit(smem_u32(&sm.bar_drain[1]));
+    mbar_wait_drain(smem_u32(&sm.bar_drain[1]), 0, status_word, 2);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ dS (2 threads / row)
     const int ew = threadIdx.x - 128;
@@ -352,6 +357,7 @@ struct DkvSmem {
   uint64_t bar_do_full[kDoStages], bar_do_empty[kDoStages];
   uint64_t bar_s_full, bar_x_free, bar_dp_full, bar_pds_full;
   uint64_t bar_acc_done;
+  uint64_t bar_drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -442,6 +448,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     mbar_init(b_dp, 1);
     mbar_init(b_pds, kDkvElem);
     mbar_init(b_acc, 1);
+    mbar_init(smem_u32(&sm.bar_drain), 1);
     sm.abort_flag = 0;
     mbar_fence_init();
   }
@@ -503,12 +510,10 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     }
     // no copy may still be writing shared memory when the CTA exits
     for (int c = (q_issued > kQStages ? q_issued - kQStages : 0); c < q_issued; ++c)
-      mbar_wait(smem_u32(&sm.bar_q_full[c % kQStages]), (c / kQStages) & 1, abort_flag,
-                status_word, 2);
+      mbar_wait_drain(smem_u32(&sm.bar_q_full[c % kQStages]), (c / kQStages) & 1, status_word, 2);
     for (int c = (do_issued > kDoStages ? do_issued - kDoStages : 0); c < do_issued; ++c)
-      mbar_wait(smem_u32(&sm.bar_do_full[c % kDoStages]), (c / kDoStages) & 1, abort_flag,
-                status_word, 2);
-    if (total > 0) mbar_wait(b_kv, 0, abort_flag, status_word, 2);
+      mbar_wait_drain(smem_u32(&sm.bar_do_full[c % kDoStages]), (c / kDoStages) & 1, status_word, 2);
+    if (total > 0) mbar_wait_drain(b_kv, 0, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     // Issue order per chunk c: S^T(c+1), dK(c), dV(c), dP^T(c+1).  S^T(c+1)
@@ -578,6 +583,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       else if (c + 1 < total && !issue_dp(c + 1)) ok = false;
     }
     if (ok && total > 0) mma_commit(b_acc);
+    mma_commit(smem_u32(&sm.bar_drain));
+    mbar_wait_drain(smem_u32(&sm.bar_drain), 0, status_word, 2);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ P^T, dS^T (4 threads / key)
     const int qq = (warp - 2) >> 2;   // query quarter: [32 qq, 32 qq + 32)
@@ -701,7 +708,8 @@ ba_status launch_kernel(K kernel, size_t smem, int64_t grid, int threads, const 
 
 }  // namespace
 
-bool sm100_bwd_available() { return true; }
+bool sm100_fused_bwd_available() { return false; }
+ba_status launch_bwd_fused_sm100(const AttnParams &, cudaStream_t) { return BA_ERR_UNSUPPORTED; }
 
 ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s) {
   const int d = a.head_dim;

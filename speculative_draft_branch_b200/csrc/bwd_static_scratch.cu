@@ -5,16 +5,17 @@
 // pool at start-up, or a plugin whose host forbids allocation once it is
 // running.  Such callers cannot cudaMalloc the backward workspace that
 // branch_attn_bwd asks for.  This entry point runs the same backward with its
-// scratch (D = rowsum(dO * O) plus the fp32 dQ accumulator or the per-query
-// records) placed in a file-scope device array instead, so it allocates
+// scratch (D = rowsum(dO * O), the per-query records and the fp32 dQ
+// accumulator) placed in a file-scope device array instead, so it allocates
 // nothing.
 //
 // The array is a module global: every GPU that loads this library holds
 // kStaticScratchBytes of it until the process exits.  All calls on a device
 // share that one array and it keeps whatever the last call left in it; the
-// backward rewrites D and the records (or zeroes the dQ accumulator) itself on
-// every call, so nothing has to be cleared in between.  Two calls whose kernels overlap on
-// the GPU (different streams without ordering) race on the array.
+// backward rewrites D and the records on every call, and the fused backward
+// zeroes its dQ accumulator before it sums into it, so nothing has to be
+// cleared in between.  Two calls whose kernels overlap on the GPU (different
+// streams without ordering) race on the array.
 #include <mutex>
 
 #include "internal.cuh"
@@ -31,9 +32,30 @@ static __device__ __align__(256) unsigned char g_bwd_scratch[kStaticScratchBytes
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_addr[kMaxDevices] = {};
+void *g_ctx[kMaxDevices] = {};  // the context g_addr[dev] was looked up in
 
-// Device address of the scratch array on the current device; looked up once
-// per device (with that device current) and cached.
+using CtxGetCurrentFn = int (*)(void **);
+
+// The driver's cuCtxGetCurrent, found through the runtime (the library links
+// no driver library); null if the driver does not provide it.
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of the scratch array on the current device, looked up with
+// that device current once per device context and cached.  The cache is keyed
+// on the context as well as the device ordinal, so after a device reset (a new
+// primary context) the address is looked up again instead of reusing one that
+// belonged to the destroyed context.
 ba_status scratch_address(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -42,12 +64,25 @@ ba_status scratch_address(void **out) {
     set_error("device %d outside the supported range for the static scratch", dev);
     return BA_ERR_UNSUPPORTED;
   }
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) {
+    set_error("cuCtxGetCurrent unavailable: cannot key the static scratch address on a context");
+    return BA_ERR_CUDA;
+  }
+  void *ctx = nullptr;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
+  if (get(&ctx) != 0 || !ctx || !g_addr[dev] || g_ctx[dev] != ctx) {
+    // the runtime call binds the device's primary context to this thread if
+    // none is current yet; the context is read again after it
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_bwd_scratch);
     if (e != cudaSuccess) return cuda_check(e, "cudaGetSymbolAddress(static backward scratch)");
+    if (get(&ctx) != 0 || !ctx) {
+      set_error("no CUDA context is current after the static scratch lookup");
+      return BA_ERR_CUDA;
+    }
     g_addr[dev] = p;
+    g_ctx[dev] = ctx;
   }
   *out = g_addr[dev];
   return BA_OK;

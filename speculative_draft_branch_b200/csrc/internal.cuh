@@ -40,7 +40,7 @@ struct AttnParams {
   float *dq_acc;              // [(N + Nb), Hq, d] fp32
   __nv_bfloat16 *dk_m, *dv_m, *dk_b, *dv_b;
   __nv_bfloat16 *dq_out_m, *dq_out_b;  // dQ written directly (tcgen05 backward)
-  int32_t zero_dq_acc;                  // preprocess clears dq_acc (mma.sync backward)
+  int32_t zero_dq_acc;                  // preprocess clears dq_acc
   // per-query backward records {LSE * log2(e), D, key lo, key hi} (tcgen05
   // backward): rec[kind][h][padded row], kind 0 = main-key interval, 1 =
   // branch-local interval; main rows at [0, n_main_pad), branch rows after.
@@ -77,15 +77,11 @@ ba_status launch_dq_convert(const AttnParams &a, __nv_bfloat16 *dq_m, __nv_bfloa
                             cudaStream_t s);
 ba_status launch_zz_finalize(const AttnParams &a, cudaStream_t s);
 
-// mma.sync kernels (pre-Blackwell tensor-core path)
-ba_status launch_fwd_mma(const AttnParams &a, cudaStream_t s);
-ba_status launch_bwd_mma(const AttnParams &a, cudaStream_t s);
 // tcgen05 / TMEM / TMA kernels
-bool sm100_available();
-bool sm100_fwd_available();
-bool sm100_bwd_available();
 ba_status launch_fwd_sm100(const AttnParams &a, cudaStream_t s);
 ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s);
+bool sm100_fused_bwd_available();
+ba_status launch_bwd_fused_sm100(const AttnParams &a, cudaStream_t s);
 ba_status launch_exp2_check(const float *x, float *y_fma, float *y_mufu, int64_t n,
                             cudaStream_t s);
 

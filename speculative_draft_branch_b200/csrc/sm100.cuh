@@ -69,6 +69,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Wait used when a CTA tears down: for copies or MMAs it has already issued,
+// so that nothing still writes its shared memory or TMEM when it frees them
+// and exits.  Ignores the abort flag (those operations complete whether or
+// not the CTA aborted) and gives up only after the same time limit, setting
+// the status bit of `where` then.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, int *status_word,
+                                                int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15) == 0 && global_ns() - t0 > kWaitNs) {
+      atomicOr(status_word, 1 << (where & 15));
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");

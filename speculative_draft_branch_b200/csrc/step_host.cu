@@ -184,21 +184,34 @@ extern "C" ba_status branch_attn_step_host(
     return bytes ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, c->down)
                  : cudaSuccess;
   };
+  // Once a copy is queued it reads or writes the caller's host buffers.  An
+  // error after that point waits for every copy already queued on the two
+  // copy streams before returning, so the caller may reuse its buffers as soon
+  // as the call has returned, whatever the outcome.
+  bool queued = false;
+  auto settle = [&](ba_status st_err) {
+    if (queued) {
+      cudaStreamSynchronize(c->up);
+      cudaStreamSynchronize(c->down);
+    }
+    return st_err;
+  };
 #define BA_TRY(x)                                                  \
   do {                                                             \
     cudaError_t e_ = (x);                                          \
-    if (e_ != cudaSuccess) return cuda_check(e_, #x);              \
+    if (e_ != cudaSuccess) return settle(cuda_check(e_, #x));      \
   } while (0)
 #define BA_TRY_ST(x)                     \
   do {                                   \
     ba_status s_ = (x);                  \
-    if (s_ != BA_OK) return s_;          \
+    if (s_ != BA_OK) return settle(s_);  \
   } while (0)
 
   // uploads wait for the caller's earlier work on `stream` (which may still
   // read this staging area)
   BA_TRY(cudaEventRecord(c->start, stream));
   BA_TRY(cudaStreamWaitEvent(c->up, c->start, 0));
+  queued = true;
   BA_TRY(h2d(d_cu, p->cu_seqlens, s.cu));
   BA_TRY(h2d(d_anchor, p->branch_anchor, s.anchor));
   BA_TRY(h2d(d_depth, p->branch_depth, s.depth));

@@ -66,7 +66,7 @@ int main(void) {
   if (ba_wait_check(NULL, 0, NULL) != BA_ERR_INVALID_ARG) return failed("wait check without a plan");
   if (lse_merge(0, 4, 64, 1, NULL, NULL, NULL, NULL, NULL, NULL, NULL) != BA_OK)
     return failed("empty merge is a no-op");
-  if (ba_set_kernel_family(3) != BA_ERR_INVALID_ARG) return failed("unknown kernel family");
+  if (ba_set_kernel_family(2) != BA_ERR_INVALID_ARG) return failed("unknown kernel family");
 
   printf("ok\n");
   return 0;

@@ -43,36 +43,43 @@ def test_hbm_steps_byte_accounting(monkeypatch):
         calls["merge"] += 1
 
     def set_events(which, start=None, stop=None):
-        assert which == 1
+        assert which == 2                          # the preprocess kernel's own events
         calls["events"].append(start is not None)
         ks_ke["pair"] = (start, stop)
 
-    ba = types.SimpleNamespace(lse_merge=lse_merge, ba_set_kernel_events=set_events)
+    ba = types.SimpleNamespace(lse_merge=lse_merge, ba_set_kernel_events=set_events,
+                               ba_get_kernel_family=lambda: family[0])
 
     class Runner:
         problem = types.SimpleNamespace(c=types.SimpleNamespace(
             n_main=1000, n_branch_tokens=3000, hq=4, head_dim=64))
 
         def backward(self, t, out, grads):
-            # the library records its kernel events around the attention kernels
+            # the library records the preprocess events right around its kernel
             calls["bwd"] += 1
             start, stop = ks_ke["pair"]
             start.record()
+            _Clock.t += 1.0                       # the kernel itself: 2 ticks apart
             stop.record()
 
-    res = bench.hbm_steps(ba, Runner(), {}, {}, {}, None, "cpu", hbm_gbs=1000.0, max_rows=2500)
-    assert calls["merge"] == 13 and calls["bwd"] == 5
-    assert calls["events"][-1] is False           # events switched off afterwards
-    m = res["lse_merge"]
-    assert m["rows"] == 2500                      # capped at max_rows
-    assert m["bytes_per_launch"] == 2500 * 4 * (3 * 64 * 4 + 3 * 4)
-    assert m["ms"] == pytest.approx(0.1)          # 10 calls between two ticks
-    p = res["bwd_preprocess"]
-    # call span c0 -> c1 is 3 ticks (kernel start, kernel stop, end), kernel span 1 tick
-    assert p["ms"] == pytest.approx(2.0)
-    assert p["bytes_per_launch"] == 4000 * 4 * (2 * 64 * 2 + 4 + 4 + 32) + 4000 * 16
-    assert p["frac"] == pytest.approx(p["achieved"] / 1000.0)
-    assert p["achieved"] == pytest.approx(p["bytes_per_launch"] / 2e-3 / 1e9)
+    for fam, zero in ((1, 0), (0, 4 * 64)):
+        family = [fam]
+        calls.update(merge=0, bwd=0, events=[])
+        res = bench.hbm_steps(ba, Runner(), {}, {}, {}, None, "cpu", hbm_gbs=1000.0,
+                              max_rows=2500)
+        assert calls["merge"] == 13 and calls["bwd"] == 5
+        assert calls["events"][-1] is False           # events switched off afterwards
+        m = res["lse_merge"]
+        assert m["rows"] == 2500                      # capped at max_rows
+        assert m["bytes_per_launch"] == 2500 * 4 * (3 * 64 * 4 + 3 * 4)
+        assert m["ms"] == pytest.approx(0.1)          # 10 calls between two ticks
+        p = res["bwd_preprocess"]
+        assert p["ms"] == pytest.approx(2.0)
+        # O, dO, LSE read, D and two records written per row-head (plus the zeroed
+        # fp32 dQ accumulator of the fused backward), key interval read per row
+        assert p["bytes_per_launch"] == 4000 * 4 * (2 * 64 * 2 + 4 + 4 + 32 + zero) + 4000 * 16
+        assert p["frac"] == pytest.approx(p["achieved"] / 1000.0)
+        assert p["achieved"] == pytest.approx(p["bytes_per_launch"] / 2e-3 / 1e9)
 
 
 def test_clock_sampler_parses_samples_and_reasons(monkeypatch):

@@ -258,6 +258,13 @@ def test_useful_pair_counts_closed_form():
     per = L * (L + 1) // 2 + sum(8 * (32 * k + 32) + 36 for k in range(2048))
     assert per * 32 == 85911142400
     assert oracle.useful_pairs(wl.structure("dspark_64k")) == 85911142400
+    # TTT 256K: one sequence, depth-3 TTT-causal branch at every position:
+    # main L(L+1)/2; branch at p sees p+1 main keys at each of its 3 depths
+    # (3 L(L+1)/2) plus 1+2+3 = 6 branch keys, x 32 heads
+    L = 262144
+    per = L * (L + 1) // 2 + 3 * L * (L + 1) // 2 + 6 * L
+    assert per * 32 == 4398113619968
+    assert oracle.useful_pairs(wl.structure("ttt_256k")) == 4398113619968
 
 
 def test_useful_pairs_match_dense_mask():
@@ -407,3 +414,33 @@ def test_zz_tiles_cover_every_ring_step_pair():
                 for k in keys:
                     assert zz[step, t, 2 * w] <= k // BM < zz[step, t, 2 * w + 1]
         np.testing.assert_array_equal(seen, mask[r, :n].astype(int))
+
+
+# ---------------------------------------------------------- zero queries (closed form)
+@pytest.mark.parametrize("kind", KINDS)
+def test_visible_counts_match_dense_mask(kind):
+    st = wl.random_structure(17, n_seqs=3, max_len=40, max_depth=6, mask_kind=kind)
+    n_m, n_b = oracle.visible_counts(st)
+    rows = oracle.dense_mask(st).sum(axis=1)
+    np.testing.assert_array_equal(np.concatenate([n_m, n_b]), rows)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("seed", [0, 1])
+def test_zero_query_dv_matches_dense_backward(kind, seed):
+    """With Q = 0 the dense backward (explicit mask, analytic gradients) gives
+    dV = the suffix-sum closed form and dK = 0, for every main and branch key."""
+    st = wl.random_structure(30 + seed, n_seqs=3, max_len=25, max_depth=5, hq=4, hkv=2,
+                             head_dim=8, mask_kind=kind, branch_prob=0.6)
+    t = _f64_tensors(st, 40 + seed)
+    t["q_m"][:] = 0.0
+    t["q_b"][:] = 0.0
+    dq_m, dk_m, dv_m, dq_b, dk_b, dv_b = oracle.backward_dense(st, t)
+    got_m, got_b = oracle.zero_query_dv(st, t)
+    np.testing.assert_allclose(got_m, dv_m, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got_b, dv_b, rtol=1e-12, atol=1e-12)
+    assert np.abs(dk_m).max() == 0.0 and np.abs(dk_b).max() == 0.0
+    # a subset of groups fills only those groups
+    part_m, part_b = oracle.zero_query_dv(st, t, groups=[1])
+    np.testing.assert_allclose(part_m[:, 1], dv_m[:, 1], rtol=1e-12, atol=1e-12)
+    assert np.abs(part_m[:, 0]).max() == 0.0 and np.abs(part_b[:, 0]).max() == 0.0
