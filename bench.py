@@ -18,8 +18,9 @@ With N > 1 (torchrun) each rank runs an independent replica of the batch
 (weak scaling: the path has no cross-GPU exchange at this layout); the step
 time is the max over ranks.  `--impl reference` times the fp64 CPU oracle on a
 bounded sample of the same workload on the host cores.  `--shard-timing C`
-(with a one-sequence workload) runs the tile-order study instead: per-shard
-times of the zigzag and the sequential order of C shards, from prefix timings.
+runs the tile-order study instead: per-shard times of the zigzag and the
+sequential order of C shards (and of C/2, C/4, ... shards), from the timings
+of packed prefixes of every sequence.
 """
 from __future__ import annotations
 
@@ -62,7 +63,8 @@ def parse_args():
                     help="skip timing the other full-size configurations after the headline")
     ap.add_argument("--shard-timing", type=int, default=0, metavar="C",
                     help="tile-order study: per-shard fwd+bwd time of the zigzag and the "
-                         "sequential order of C shards over one sequence (prints its own line)")
+                         "sequential order of C shards, C a power of two (prints its own "
+                         "line)")
     return ap.parse_args()
 
 
@@ -687,14 +689,19 @@ def shard_split(prefix, C: int):
 def run_shard_timing(args):
     """Timing half of the tile-order study, on one GPU.
 
-    One causal sequence (the workload cut to --tokens main tokens and their
-    branches) is split into 2C equal chunks.  The rows of a chunk [a, b) see
-    only keys below b, so their fwd+bwd time is T(b) - T(a), where T(x) is the
-    step time of the x-token prefix; timing the 2C prefixes that end at the
-    chunk boundaries gives every chunk's time and so every shard's, for the
-    zigzag and the sequential order.  Useful pairs come from the library's plan
-    of each prefix.  Each prefix: --warmup untimed steps, the median of --steps
-    timed ones (CUDA events on the launching stream)."""
+    Every sequence of the batch (the workload, or its first --tokens packed
+    tokens) is split into 2C equal chunks.  The rows of chunk k of a sequence
+    see only keys of chunks <= k, so the fwd+bwd time of chunk k of every
+    sequence together is T(k+1) - T(k), where T(k) is the step time of the
+    packed batch with every sequence cut to its first k chunks (and the
+    branches anchored there).  Timing those 2C packed prefixes gives every
+    chunk's time, and so every shard's, for the zigzag order (shard i: chunks
+    i and 2C-1-i of every sequence) and the sequential one (chunks 2i and
+    2i+1), for C and for every C / 2^j >= 2 as well (their chunks are unions
+    of these).  Each prefix runs in one launch over the whole packed batch, so
+    the GPU is as full as the workload makes it.  Useful pairs come from the
+    library's plan of each prefix.  Each prefix: --warmup untimed steps, the
+    median of --steps timed ones (CUDA events on the launching stream)."""
     import dataclasses
 
     import torch
@@ -706,25 +713,23 @@ def run_shard_timing(args):
     if rank != 0:
         return 0
     C = args.shard_timing
+    if C < 1 or (C & (C - 1)) != 0:
+        raise SystemExit("--shard-timing C must be a power of two")
     st_full = wl.structure(args.workload)
-    if len(st_full.cu_seqlens) != 2:
-        raise SystemExit("--shard-timing needs a one-sequence workload (ttt_256k, dspark_64k)")
-    L = args.tokens or st_full.n_main
+    base = st_full if not args.tokens else wl.truncate(st_full, args.tokens)
+    base = dataclasses.replace(base, zigzag_C=1)
     P = 2 * C
-    if C < 1 or L % (P * 128) != 0 or L > st_full.n_main:
-        raise SystemExit(f"--tokens {L} must be a multiple of 2C x 128 = {P * 128} "
-                         f"and at most {st_full.n_main}")
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    base = dataclasses.replace(wl.truncate(st_full, L), zigzag_C=1)
-    t_full = wl.tensors(base, wl.workload_seed(args.workload), dev)
+    t_base = wl.slice_tensors(st_full, base, wl.tensors(st_full, wl.workload_seed(args.workload),
+                                                        dev))
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(local_rank)
     clocks.start()
     T, pairs = [0.0], [0]
     for k in range(1, P + 1):
-        st = dataclasses.replace(wl.truncate(base, k * L // P), zigzag_C=1)
-        t = wl.slice_tensors(base, st, t_full)
+        st, mr, br = wl.truncate_each(base, k, P)
+        t = wl.gather_tensors(t_base, mr, br)
         runner = ba.BranchAttention(ba.Problem.from_structure(st, device=dev), device=dev)
         runner.plan()
         if runner.plan_status() != 0:
@@ -747,24 +752,34 @@ def run_shard_timing(args):
         del runner, out, grads, t
         torch.cuda.empty_cache()
     clk = clocks.stop()
-    tm, pr = shard_split(T, C), shard_split(pairs, C)
     d = base.head_dim
 
     def ratio(x):
         return max(x) / (sum(x) / len(x))
 
+    per_c = {}
+    c = C
+    while c >= 2:
+        step = C // c                                 # prefixes k * step of 2C
+        tm = shard_split(T[::step], c)
+        pr = shard_split(pairs[::step], c)
+        per_c[str(c)] = {
+            "zigzag": {"shard_ms": tm["zigzag"], "shard_pairs": pr["zigzag"],
+                       "max_over_mean_time": ratio(tm["zigzag"]),
+                       "max_over_mean_pairs": ratio(pr["zigzag"])},
+            "sequential": {"shard_ms": tm["sequential"], "shard_pairs": pr["sequential"],
+                           "max_over_mean_time": ratio(tm["sequential"]),
+                           "max_over_mean_pairs": ratio(pr["sequential"])}}
+        c //= 2
+    chunk_t, chunk_p = shard_split(T, C)["chunk"], shard_split(pairs, C)["chunk"]
     print(json.dumps({
-        "study": "shard_timing", "workload": args.workload, "tokens": L, "C": C,
-        "steps": args.steps, "warmup": args.warmup, "prefix_ms": T[1:],
-        "chunk_ms": tm["chunk"], "chunk_pairs": pr["chunk"],
+        "study": "shard_timing", "workload": base.name, "n_seqs": base.n_seqs,
+        "n_main": base.n_main, "n_branch_tokens": base.n_branch_tokens, "C": C,
+        "steps": args.steps, "warmup": args.warmup, "prefix_ms": T[1:], "prefix_pairs": pairs[1:],
+        "chunk_ms": chunk_t, "chunk_pairs": chunk_p,
         "chunk_tflops": [10 * d * p / (m * 1e-3) / 1e12 if m > 0 else None
-                         for p, m in zip(pr["chunk"], tm["chunk"])],
-        "zigzag": {"shard_ms": tm["zigzag"], "max_over_mean_time": ratio(tm["zigzag"]),
-                   "max_over_mean_pairs": ratio(pr["zigzag"])},
-        "sequential": {"shard_ms": tm["sequential"],
-                       "max_over_mean_time": ratio(tm["sequential"]),
-                       "max_over_mean_pairs": ratio(pr["sequential"])},
-        "clocks": clk}))
+                         for p, m in zip(chunk_p, chunk_t)],
+        "per_C": per_c, "clocks": clk}))
     return 0
 
 

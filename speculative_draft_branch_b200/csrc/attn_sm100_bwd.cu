@@ -341,7 +341,6 @@ __global__ void __launch_bounds__(384, 1)
 // ============================================================================
 // dK / dV kernel
 // ============================================================================
-constexpr int kQc = 128;      // query rows per chunk: N of the S^T / dP^T products
 constexpr int kQStages = 2;   // Q ring (freed once dK of the chunk is done)
 constexpr int kDoStages = 2;  // dO + records ring (freed once dV of the chunk is done)
 
@@ -360,33 +359,6 @@ struct DkvSmem {
   uint64_t bar_drain;
   uint32_t tmem_base;
   int abort_flag;
-};
-
-struct DkvMaps {
-  TensorMaps t;
-  CUtensorMap do_m, do_b;
-};
-
-// Chunk c of a CTA's walk: query tile step s = c / grp, q head g grp + c % grp.
-// The tile steps merge the CTA's main q tiles and branch q tiles, each taken
-// from the last down, interleaved in proportion to their counts.  Every CTA
-// of a sequence then starts on the same (highest) tiles and moves through
-// them at the same pace, so the Q / dO tiles one CTA loads are still in L2
-// when the CTAs of the other key tiles of that sequence ask for them.
-struct ChunkWalk {
-  int n_t0, n_t1, t0, t1, grp, g;
-  __device__ __forceinline__ void at(int c, const AttnParams &a, int &h, bool &is_main_q,
-                                     int &tile, int &nrows) const {
-    const int s = c / grp;
-    h = g * grp + (c - s * grp);
-    const int n = n_t0 + n_t1;
-    const int m0 = (int)((int64_t)s * n_t0 / n);
-    const int m1 = (int)((int64_t)(s + 1) * n_t0 / n);
-    is_main_q = m1 > m0;
-    tile = is_main_q ? t0 + n_t0 - 1 - m0 : t1 + n_t1 - 1 - (s - m0);
-    const int rows = is_main_q ? a.n_main : a.n_bt;
-    nrows = max(0, min(kQc, rows - tile * kQc));
-  }
 };
 
 // TMEM columns: dK [0, D), dV [D, 2D), X = S^T at 2D, Y = dP^T at 2D + 128
@@ -416,16 +388,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   const int kt = main_kv ? item : item - a.n_kt;
   const int key0 = kt * 128;
   const int n_keys = main_kv ? a.n_main : a.n_bt;
-  ChunkWalk cw;
-  cw.grp = a.hq / a.hkv;
-  cw.g = g;
-  if (main_kv) {
-    const int32_t *r = a.plan.kv_main + (int64_t)kt * 4;
-    cw.t0 = r[0]; cw.n_t0 = r[1] - r[0]; cw.t1 = r[2]; cw.n_t1 = r[3] - r[2];
-  } else {
-    const int32_t *r = a.plan.kv_branch + (int64_t)kt * 2;
-    cw.t0 = 0; cw.n_t0 = 0; cw.t1 = r[0]; cw.n_t1 = r[1] - r[0];
-  }
+  const ChunkWalk cw = make_walk(a, main_kv, kt, g);
   const int total = cw.grp * (cw.n_t0 + cw.n_t1);
   int *status_word = a.plan.status + 1;
   volatile int *abort_flag = &sm.abort_flag;
@@ -708,8 +671,6 @@ ba_status launch_kernel(K kernel, size_t smem, int64_t grid, int threads, const 
 
 }  // namespace
 
-bool sm100_fused_bwd_available() { return false; }
-ba_status launch_bwd_fused_sm100(const AttnParams &, cudaStream_t) { return BA_ERR_UNSUPPORTED; }
 
 ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s) {
   const int d = a.head_dim;

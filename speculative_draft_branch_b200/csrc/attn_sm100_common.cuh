@@ -69,4 +69,50 @@ __device__ __forceinline__ TileSegs make_segs(const AttnParams &a, int t, bool i
   return ts;
 }
 
+
+// ---- key-stationary backward walk -------------------------------------------
+constexpr int kQc = 128;  // query rows per chunk: N of the S^T / dP^T products
+
+struct DkvMaps {
+  TensorMaps t;
+  CUtensorMap do_m, do_b;
+};
+
+// Chunk c of a CTA's walk: query tile step s = c / grp, q head g grp + c % grp.
+// The tile steps merge the CTA's main q tiles and branch q tiles, each taken
+// from the last down, interleaved in proportion to their counts.  Every CTA
+// of a sequence then starts on the same (highest) tiles and moves through
+// them at the same pace, so the Q / dO tiles one CTA loads are still in L2
+// when the CTAs of the other key tiles of that sequence ask for them.
+struct ChunkWalk {
+  int n_t0, n_t1, t0, t1, grp, g;
+  __device__ __forceinline__ void at(int c, const AttnParams &a, int &h, bool &is_main_q,
+                                     int &tile, int &nrows) const {
+    const int s = c / grp;
+    h = g * grp + (c - s * grp);
+    const int n = n_t0 + n_t1;
+    const int m0 = (int)((int64_t)s * n_t0 / n);
+    const int m1 = (int)((int64_t)(s + 1) * n_t0 / n);
+    is_main_q = m1 > m0;
+    tile = is_main_q ? t0 + n_t0 - 1 - m0 : t1 + n_t1 - 1 - (s - m0);
+    const int rows = is_main_q ? a.n_main : a.n_bt;
+    nrows = max(0, min(kQc, rows - tile * kQc));
+  }
+};
+
+// The CTA's walk for (key tile item of the plan's backward order, kv head g).
+__device__ __forceinline__ ChunkWalk make_walk(const AttnParams &a, bool main_kv, int kt, int g) {
+  ChunkWalk cw;
+  cw.grp = a.hq / a.hkv;
+  cw.g = g;
+  if (main_kv) {
+    const int32_t *r = a.plan.kv_main + (int64_t)kt * 4;
+    cw.t0 = r[0]; cw.n_t0 = r[1] - r[0]; cw.t1 = r[2]; cw.n_t1 = r[3] - r[2];
+  } else {
+    const int32_t *r = a.plan.kv_branch + (int64_t)kt * 2;
+    cw.t0 = 0; cw.n_t0 = 0; cw.t1 = r[0]; cw.n_t1 = r[1] - r[0];
+  }
+  return cw;
+}
+
 }  // namespace ba

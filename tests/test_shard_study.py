@@ -100,3 +100,43 @@ def test_prefix_differences_give_the_shard_totals(C):
         np.testing.assert_array_equal(split[order], ss.pair_matrix(base, C, order).sum(axis=1))
     with pytest.raises(ValueError):
         bench.shard_split(prefix[:-1], C)
+
+
+@pytest.mark.parametrize("name", ["ttt_20k", "dflash_32k"])
+def test_packed_prefix_differences_give_the_shard_totals(name):
+    """The packed-batch form of the same decomposition: every sequence cut to
+    its first k of 2C chunks (workloads.truncate_each); the differences of the
+    prefixes' pair counts, split by bench.shard_split, equal the pair matrix's
+    shard totals for both orders, for C = 8 and for C = 4, 2 from every second
+    or fourth prefix (the subsampling bench.py's shard timing uses)."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    st = wl.structure(name)
+    C = 8
+    prefix = [0] + [oracle.useful_pairs(wl.truncate_each(st, k, 2 * C)[0])
+                    for k in range(1, 2 * C + 1)]
+    assert prefix[-1] == oracle.useful_pairs(st)
+    for c in (8, 4, 2):
+        split = bench.shard_split(prefix[::C // c], c)
+        for order in ss.ORDERS:
+            np.testing.assert_array_equal(split[order], ss.pair_matrix(st, c, order).sum(axis=1))
+
+
+def test_truncate_each_keeps_rows_and_branches():
+    st = wl.random_structure(5, n_seqs=4, max_len=50, max_depth=4, branch_prob=0.5)
+    sub, mr, br = wl.truncate_each(st, 3, 8)
+    lens = np.diff(st.cu_seqlens)
+    kept = (3 * lens) // 8
+    assert sub.n_main == kept.sum() == len(mr)
+    assert sub.n_branch_tokens == len(br)
+    # the kept branches are exactly those anchored in kept rows, in order, with
+    # their anchors re-indexed into the kept rows and their own rows gathered
+    sel = np.nonzero(np.isin(st.anchors, mr))[0]
+    np.testing.assert_array_equal(mr[sub.anchors], st.anchors[sel])
+    np.testing.assert_array_equal(sub.depths, st.depths[sel])
+    dv = oracle.derive(st)
+    rows = [np.arange(dv.cu_branch[b], dv.cu_branch[b + 1]) for b in sel]
+    np.testing.assert_array_equal(br, np.concatenate(rows) if rows else np.zeros(0, int))
+    assert np.all(np.diff(sub.cu_seqlens) > 0)

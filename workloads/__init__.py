@@ -186,3 +186,40 @@ def slice_tensors(st_full: Structure, st_trunc: Structure, t: dict) -> dict:
     for key, x in t.items():
         out[key] = x[:n] if key.endswith("_m") else x[:nb]
     return out
+
+
+def truncate_each(st: Structure, k: int, parts: int):
+    """Every sequence of a batch cut to its first floor(k L / parts) tokens (L its
+    length; sequences cut to nothing are dropped) with the branches anchored in
+    what is kept.  Returns the structure and the kept main rows and branch rows
+    of the original batch, in order, for gather_tensors."""
+    cu = st.cu_seqlens
+    lens = np.diff(cu)
+    keep_len = (k * lens) // parts
+    main_rows, new_cu = [], [0]
+    for s in range(st.n_seqs):
+        if keep_len[s] > 0:
+            main_rows.append(np.arange(cu[s], cu[s] + keep_len[s]))
+            new_cu.append(new_cu[-1] + int(keep_len[s]))
+    main_rows = np.concatenate(main_rows) if main_rows else np.zeros(0, dtype=np.int64)
+    new_index = np.full(st.n_main, -1, dtype=np.int64)
+    new_index[main_rows] = np.arange(main_rows.shape[0])
+    cu_branch = np.concatenate([[0], np.cumsum(st.depths)])
+    sel = np.nonzero(new_index[st.anchors] >= 0)[0] if st.n_branches else np.zeros(0, np.int64)
+    branch_rows = (np.concatenate([np.arange(cu_branch[b], cu_branch[b + 1]) for b in sel])
+                   if sel.size else np.zeros(0, dtype=np.int64))
+    out = dataclasses.replace(st, name=f"{st.name}[{k}/{parts} of each sequence]",
+                              cu_seqlens=np.asarray(new_cu, dtype=np.int64),
+                              anchors=new_index[st.anchors[sel]], depths=st.depths[sel])
+    return out, main_rows, branch_rows
+
+
+def gather_tensors(t: dict, main_rows, branch_rows) -> dict:
+    """Rows of a batch's tensors picked by truncate_each (contiguous copies)."""
+    import torch
+    out = {}
+    for key, x in t.items():
+        rows = main_rows if key.endswith("_m") else branch_rows
+        idx = torch.as_tensor(np.asarray(rows, dtype=np.int64), device=x.device)
+        out[key] = x.index_select(0, idx).contiguous()
+    return out
