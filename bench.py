@@ -59,6 +59,8 @@ def parse_args():
                     help="profile-sized case: only the first N main tokens and their branches")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--family", type=int, default=0, choices=(0, 1),
+                    help="backward kernel family: 0 split (default), 1 fused")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip timing the other full-size configurations after the headline")
     ap.add_argument("--shard-timing", type=int, default=0, metavar="C",
@@ -311,7 +313,7 @@ def hbm_steps(ba, runner, t, out, grads, stream, dev, hbm_gbs, max_rows=1 << 18)
     kernels; the library records a pair of CUDA events right around it.  Per
     (row, head) it reads O and dO (2 d bf16) and the LSE and writes D and two
     16-byte records; per row it reads the 16-byte key interval; with the fused
-    backward (family 0) it also zeroes the fp32 dQ accumulator, 4 d bytes per
+    backward (family 1) it also zeroes the fp32 dQ accumulator, 4 d bytes per
     row and head."""
     import torch
     c = runner.problem.c
@@ -361,7 +363,7 @@ def hbm_steps(ba, runner, t, out, grads, stream, dev, hbm_gbs, max_rows=1 << 18)
                 times.append(ps.elapsed_time(pe))
     finally:
         ba.ba_set_kernel_events(2, None, None)
-    zero_acc = 4 * d if ba.ba_get_kernel_family() == 0 else 0
+    zero_acc = 4 * d if ba.ba_get_kernel_family() == 1 else 0
     res["bwd_preprocess"] = roof(rows * heads * (2 * d * 2 + 4 + 4 + 32 + zero_acc) + rows * 16,
                                  statistics.median(times),
                                  note="CUDA events on the launching stream around the "
@@ -466,6 +468,7 @@ def run_ours(args):
     rank, world, local_rank = rank_info()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    ba.ba_set_kernel_family(args.family)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),

@@ -290,14 +290,17 @@ BA_API ba_status ba_exp2_check(const float *x, float *y_fma, float *y_hw, int64_
 BA_API ba_status ba_wait_check(void *plan_ws, int32_t arrive, ba_stream_t stream);
 
 /* Backward kernel family (the forward is the same for both):
- *   0 = default: one fused tcgen05 kernel per (key tile, kv head) computing
+ *   0 = default: split backward, a key-stationary dK/dV kernel and a
+ *       query-stationary dQ kernel (S and dP computed in both, seven tile
+ *       products), every gradient written once in bf16; bit-reproducible
+ *       from run to run;
+ *   1 = fused backward: one tcgen05 kernel per (key tile, kv head) computing
  *       S, dP, dV, dK and dQ (the method's five tile products); dQ partials
  *       are summed in fp32 in the workspace and converted to bf16 by a final
  *       pass, so dQ may differ in the last bits from run to run (the order of
- *       the fp32 sums is not fixed); dK and dV are deterministic;
- *   1 = split backward: a key-stationary dK/dV kernel and a query-stationary
- *       dQ kernel (S and dP computed twice, seven tile products), every
- *       gradient written once in bf16; bit-reproducible from run to run.
+ *       the fp32 sums is not fixed).  It moves 64 KB of fp32 partials into L2
+ *       per (key tile, query tile, head), which on B200 makes it slower than
+ *       family 0 at head_dim 128.
  * Returns BA_ERR_INVALID_ARG for other values.  Process-wide. */
 BA_API ba_status ba_set_kernel_family(int32_t family);
 BA_API int32_t ba_get_kernel_family(void);

@@ -17,6 +17,6 @@ Parity pins for every function live in tests/test_oracle_*.py.
 from .branch_attention import (  # noqa: F401
     Derived, derive, visible_keys, dense_mask, forward_dense, backward_dense,
     lse_merge, split_forward, zigzag_chunks, zigzag_forward, rows_forward,
-    rows_backward_dq, keys_backward, useful_pairs, to64, visible_counts, zero_query_dv,
+    rows_backward_dq, keys_backward, keys_backward_both, useful_pairs, to64, visible_counts, zero_query_dv, round_bf16,
 )
 from .plan import plan, row_intervals, PLAN_BM, PLAN_BN  # noqa: F401

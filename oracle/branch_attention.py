@@ -407,7 +407,14 @@ def rows_backward_dq(st, t, main_rows=(), branch_rows=(), heads=None):
     return rows_forward(st, t, main_rows, branch_rows, with_dq=True, heads=heads)
 
 
-def keys_backward(st, t, main_keys=(), branch_keys=(), groups=None):
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """x rounded to the nearest bf16 value (ties to even), back in fp64."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)).to(
+        torch.bfloat16).to(torch.float64).numpy()
+
+
+def keys_backward(st, t, main_keys=(), branch_keys=(), groups=None, operand_bf16=False):
     """dK and dV of selected key rows, summed over every query that sees them.
 
     P_ik = exp(S_ik - l_i) needs only q_i, k and the query's LSE l_i, which
@@ -417,7 +424,22 @@ def keys_backward(st, t, main_keys=(), branch_keys=(), groups=None):
     Returns dict with dk_m/dv_m [len(main_keys), Hkv, d] and dk_b/dv_b
     [len(branch_keys), Hkv, d]; only kv heads in `groups` (default: all) are
     computed, each summed over all q heads of its group.
+
+    operand_bf16=True rounds P and dS to bf16 before they multiply dO and q
+    (everything else stays fp64): the precision in which a bf16 tensor-core
+    product receives them, so that a kernel's error can be separated from what
+    the rounding of those operands alone causes.
     """
+    return _keys_backward(st, t, main_keys, branch_keys, groups, (bool(operand_bf16),))[0]
+
+
+def keys_backward_both(st, t, main_keys=(), branch_keys=(), groups=None):
+    """keys_backward in fp64 and with bf16 operands, sharing the row forward:
+    returns (exact, bf16_operands)."""
+    return tuple(_keys_backward(st, t, main_keys, branch_keys, groups, (False, True)))
+
+
+def _keys_backward(st, t, main_keys, branch_keys, groups, modes):
     dv = derive(st)
     hq, hkv, d = st.hq, st.hkv, st.head_dim
     grp = hq // hkv
@@ -458,23 +480,23 @@ def keys_backward(st, t, main_keys=(), branch_keys=(), groups=None):
     vm_sel = to64(t["v_m"][main_keys]) if main_keys.size else np.zeros((0, hkv, d))
     kb_sel = to64(t["k_b"][branch_keys]) if branch_keys.size else np.zeros((0, hkv, d))
     vb_sel = to64(t["v_b"][branch_keys]) if branch_keys.size else np.zeros((0, hkv, d))
-    dk_m = np.zeros((main_keys.size, hkv, d))
-    dv_m = np.zeros((main_keys.size, hkv, d))
-    dk_b = np.zeros((branch_keys.size, hkv, d))
-    dv_b = np.zeros((branch_keys.size, hkv, d))
+    res = [{"dk_m": np.zeros((main_keys.size, hkv, d)), "dv_m": np.zeros((main_keys.size, hkv, d)),
+            "dk_b": np.zeros((branch_keys.size, hkv, d)), "dv_b": np.zeros((branch_keys.size, hkv, d))}
+           for _ in modes]
     for h in heads:
         g = h // grp
         dd = (dox[:, h] * fw["o"][:, h]).sum(axis=1)                # D_i = dO_i . O_i
-        for vis, ksel, vsel, dk, dvv in ((vis_m, km_sel, vm_sel, dk_m, dv_m),
-                                         (vis_b, kb_sel, vb_sel, dk_b, dv_b)):
+        for vis, ksel, vsel, kind in ((vis_m, km_sel, vm_sel, "m"), (vis_b, kb_sel, vb_sel, "b")):
             if ksel.shape[0] == 0:
                 continue
             s_ik = st.scale * (qx[:, h] @ ksel[:, g].T)             # [R, keys]
             p = np.where(vis, np.exp(np.where(vis, s_ik, 0.0) - fw["lse"][h][:, None]), 0.0)
             ds = p * (dox[:, h] @ vsel[:, g].T - dd[:, None])
-            dvv[:, g] += p.T @ dox[:, h]
-            dk[:, g] += st.scale * (ds.T @ qx[:, h])
-    return {"dk_m": dk_m, "dv_m": dv_m, "dk_b": dk_b, "dv_b": dv_b}
+            for out, rounded in zip(res, modes):
+                pp, dss = (round_bf16(p), round_bf16(ds)) if rounded else (p, ds)
+                out["dv_" + kind][:, g] += pp.T @ dox[:, h]
+                out["dk_" + kind][:, g] += st.scale * (dss.T @ qx[:, h])
+    return res
 
 
 def useful_pairs(st) -> int:

@@ -379,10 +379,10 @@ ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws, void *bwd_ws
   a.dq_out_m = (__nv_bfloat16 *)dq_m;
   a.dq_out_b = (__nv_bfloat16 *)dq_b;
   cudaStream_t s = (cudaStream_t)stream;
-  // family 0: one fused kernel accumulating dQ in fp32 (the preprocess zeroes
-  // the accumulator, a last pass converts it); family 1: the deterministic
-  // split backward (dK/dV kernel + dQ kernel, both writing bf16 directly)
-  const bool fused = g_family.load() == 0 && sm100_fused_bwd_available();
+  // family 0: the split backward (dK/dV kernel + dQ kernel, both writing bf16
+  // directly; deterministic); family 1: one fused kernel accumulating dQ in
+  // fp32 (the preprocess zeroes the accumulator, a last pass converts it)
+  const bool fused = g_family.load() == 1 && sm100_fused_bwd_available();
   a.zero_dq_acc = fused ? 1 : 0;
   record_event(2, true, s);
   BA_TRY(launch_bwd_preprocess(a, s));

@@ -62,7 +62,7 @@ def test_hbm_steps_byte_accounting(monkeypatch):
             _Clock.t += 1.0                       # the kernel itself: 2 ticks apart
             stop.record()
 
-    for fam, zero in ((1, 0), (0, 4 * 64)):
+    for fam, zero in ((0, 0), (1, 4 * 64)):
         family = [fam]
         calls.update(merge=0, bwd=0, events=[])
         res = bench.hbm_steps(ba, Runner(), {}, {}, {}, None, "cpu", hbm_gbs=1000.0,

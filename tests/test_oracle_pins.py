@@ -444,3 +444,50 @@ def test_zero_query_dv_matches_dense_backward(kind, seed):
     part_m, part_b = oracle.zero_query_dv(st, t, groups=[1])
     np.testing.assert_allclose(part_m[:, 1], dv_m[:, 1], rtol=1e-12, atol=1e-12)
     assert np.abs(part_m[:, 0]).max() == 0.0 and np.abs(part_b[:, 0]).max() == 0.0
+
+
+# ---------------------------------------------------------- bf16 operand model
+def test_round_bf16_is_round_to_nearest_even():
+    # values on the bf16 grid stay; midpoints go to the even neighbour
+    assert oracle.round_bf16(np.array([1.0, 1.0 + 2 ** -7]))[1] == 1.0 + 2 ** -7
+    assert oracle.round_bf16(np.array([1.0 + 2 ** -8]))[0] == 1.0          # tie -> even
+    assert oracle.round_bf16(np.array([1.0 + 3 * 2 ** -8]))[0] == 1.0 + 2 ** -6
+    x = np.random.default_rng(0).standard_normal(1000)
+    r = oracle.round_bf16(x)
+    assert np.all(np.abs(r - x) <= np.abs(x) * 2 ** -8)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_keys_backward_with_bf16_operands_matches_dense(kind):
+    """operand_bf16=True equals the dense definition with P and dS rounded to
+    bf16 (explicit mask, union softmax, dense products)."""
+    st = wl.random_structure(23, n_seqs=2, max_len=20, max_depth=4, hq=4, hkv=2, head_dim=8,
+                             mask_kind=kind, branch_prob=0.6)
+    t = _f64_tensors(st, 5)
+    dvr = oracle.derive(st)
+    mask = oracle.dense_mask(st, dvr)
+    n = dvr.n_main
+    q = np.concatenate([t["q_m"], t["q_b"]])
+    k = np.concatenate([t["k_m"], t["k_b"]])
+    v = np.concatenate([t["v_m"], t["v_b"]])
+    do = np.concatenate([t["do_m"], t["do_b"]])
+    grp = st.hq // st.hkv
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for h in range(st.hq):
+        g = h // grp
+        s = st.scale * q[:, h] @ k[:, g].T
+        s = np.where(mask, s, -np.inf)
+        lse = np.log(np.exp(s - s.max(1, keepdims=True)).sum(1)) + s.max(1)
+        p = np.where(mask, np.exp(s - lse[:, None]), 0.0)
+        o = p @ v[:, g]
+        ds = p * (do[:, h] @ v[:, g].T - (do[:, h] * o).sum(1)[:, None])
+        dv[:, g] += oracle.round_bf16(p).T @ do[:, h]
+        dk[:, g] += st.scale * oracle.round_bf16(ds).T @ q[:, h]
+    mk = list(range(n))
+    bk = list(range(dvr.n_branch_tokens))
+    got = oracle.keys_backward(st, t, mk, bk, operand_bf16=True)
+    np.testing.assert_allclose(got["dv_m"], dv[:n], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got["dk_m"], dk[:n], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got["dv_b"], dv[n:], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got["dk_b"], dk[n:], rtol=1e-12, atol=1e-12)
