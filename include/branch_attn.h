@@ -267,6 +267,79 @@ BA_API ba_status lse_merge(int64_t rows, int32_t heads, int32_t head_dim,
                     const void *o_b, const float *lse_b, void *o_out,
                     float *lse_out, ba_stream_t stream);
 
+/* ---- Zigzag context parallelism across ranks --------------------------------
+ * The core-innovation and method-detail sections shard a packed batch over C
+ * context-parallel ranks in zigzag order and send the main-sequence K/V round
+ * a ring: every sequence of length L is cut into 2C chunks, chunk k covering
+ * positions [floor(kL/2C), floor((k+1)L/2C)); shard q holds chunks q and
+ * 2C-1-q of every sequence and the branches anchored in them (branch K/V never
+ * leave their rank).  At ring step t the rank holding shard q attends its
+ * queries to the main keys of shard (q - t) mod C and merges the step's
+ * partial (O, l) into an fp32 accumulator by the LSE rule; the rank-local
+ * branch keys are merged last.  A shard is kept as its own packed problem
+ * (the "local" problem): per sequence, its two chunks in position order.
+ * Every sequence must hold at least 2C tokens. */
+
+/* Host-only: the local problem of one shard.  cu_seqlens [n_seqs + 1],
+ * branch_anchor and branch_depth [n_branches] are HOST arrays of the whole
+ * batch (anchors non-decreasing).  Writes the shard's sizes to the three
+ * count pointers and, for every output pointer that is not NULL (host arrays
+ * sized by those counts): cu_local [n_seqs + 1] (local cu_seqlens: every
+ * sequence keeps its index), anchor_local / depth_local [n_branches_local]
+ * (anchors as local main rows), main_rows [n_main_local] (the batch's main
+ * row of each local main row) and branch_rows [n_branch_tokens_local] (the
+ * batch's branch row of each local branch row).  BA_ERR_UNSUPPORTED if a
+ * sequence is shorter than 2C, BA_ERR_INVALID_ARG for other bad input. */
+BA_API ba_status ba_zigzag_shard(const int32_t *cu_seqlens, int32_t n_seqs,
+                                 const int32_t *branch_anchor, const int32_t *branch_depth,
+                                 int32_t n_branches, int32_t C, int32_t shard,
+                                 int32_t *n_main_local, int32_t *n_branches_local,
+                                 int32_t *n_branch_tokens_local, int32_t *cu_local,
+                                 int32_t *anchor_local, int32_t *depth_local,
+                                 int32_t *main_rows, int32_t *branch_rows);
+
+/* Workspace sizes of a ring rank (host-only): one plan workspace per step
+ * (plan_bytes, the layout of ba_plan for the local problem) and the fp32
+ * accumulator of O and LSE for every local query row and head (acc_bytes). */
+BA_API ba_status ba_ring_workspace_size(const ba_problem *local, int32_t C, size_t *plan_bytes,
+                                        size_t *acc_bytes);
+
+/* Plan of ring step `step` (0 <= step < C) for the rank holding `shard`,
+ * against shard (shard - step) mod C.  `local` is the rank's local problem
+ * (device index arrays, zigzag_C = 1).  Step 0 is the local causal plan (the
+ * plan of ba_plan; it also carries the branch-local intervals that
+ * branch_attn_ring_finish reads).  For step > 0, cu_global [n_seqs + 1] is
+ * the whole batch's cu_seqlens and cu_visit [n_seqs + 1] the visiting shard's
+ * local cu_seqlens, both device arrays.  Async on `stream`. */
+BA_API ba_status ba_ring_plan(const ba_problem *local, int32_t C, int32_t shard, int32_t step,
+                              const int32_t *cu_global, const int32_t *cu_visit, void *plan_ws,
+                              size_t plan_bytes, ba_stream_t stream);
+
+/* One ring step: the rank's queries (q_m [n_main, Hq, d], q_b [n_branch_tokens,
+ * Hq, d] of the local problem) against the visiting shard's main K/V
+ * (k_m_visit, v_m_visit [n_main_visit, Hkv, d], in that shard's local order),
+ * with the plan of ba_plan for the same step.  Step 0 initialises the
+ * accumulator acc_ws (ba_ring_workspace_size bytes), later steps merge into it
+ * by the LSE rule.  Steps of one rank must run in order 0 .. C-1 on one
+ * stream (or be ordered by the caller).  Async on `stream`. */
+BA_API ba_status branch_attn_ring_step(const ba_problem *local, int32_t C, int32_t step,
+                                       const void *plan_ws, void *acc_ws, size_t acc_bytes,
+                                       int32_t n_main_visit, const void *q_m,
+                                       const void *k_m_visit, const void *v_m_visit,
+                                       const void *q_b, ba_stream_t stream);
+
+/* Last step: the branch-local partial of every branch query (own branch K/V,
+ * k_b / v_b of the local problem), merged into the accumulator, which then
+ * gives the outputs o_m, o_b (bf16) and lse_m, lse_b (fp32) of the local rows,
+ * in the layouts of branch_attn_fwd.  plan_ws is the step-0 plan.  The result
+ * equals branch_attn_fwd of the whole batch on the shard's rows, up to
+ * rounding. */
+BA_API ba_status branch_attn_ring_finish(const ba_problem *local, int32_t C, const void *plan_ws,
+                                         void *acc_ws, size_t acc_bytes, const void *q_m,
+                                         const void *q_b, const void *k_b, const void *v_b,
+                                         void *o_m, void *o_b, float *lse_m, float *lse_b,
+                                         ba_stream_t stream);
+
 /* Device self-check of the exponentials available to the softmax (no
  * counterpart in the paper): the hardware ex2 unit the kernels use, and a
  * range-reduced cubic on the FMA pipe (max relative error 7.5e-5) kept as an

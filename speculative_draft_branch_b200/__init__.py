@@ -32,7 +32,9 @@ EXPORTS = ("ba_workspace_size", "ba_plan_layout_query", "ba_plan", "ba_plan_stat
            "branch_attn_fwd", "branch_attn_bwd", "lse_merge", "ba_set_kernel_family",
            "ba_get_kernel_family", "ba_set_kernel_events", "ba_launch_count", "ba_last_error",
            "ba_version", "branch_attn_bwd_static_scratch", "ba_exp2_check",
-           "ba_step_host_workspace_size", "branch_attn_step_host", "ba_wait_check")
+           "ba_step_host_workspace_size", "branch_attn_step_host", "ba_wait_check",
+           "ba_zigzag_shard", "ba_ring_workspace_size", "ba_ring_plan", "branch_attn_ring_step",
+           "branch_attn_ring_finish")
 
 
 class BAProblem(ctypes.Structure):
@@ -83,6 +85,11 @@ def _load() -> ctypes.CDLL:
         "ba_wait_check": [VP, I32, VP],
         "ba_step_host_workspace_size": [P, ctypes.POINTER(S)],
         "branch_attn_step_host": [P, VP, S] + [VP] * 18 + [VP],
+        "ba_zigzag_shard": [VP, I32, VP, VP, I32, I32, I32] + [VP] * 8,
+        "ba_ring_workspace_size": [P, I32, ctypes.POINTER(S), ctypes.POINTER(S)],
+        "ba_ring_plan": [P, I32, I32, I32, VP, VP, VP, S, VP],
+        "branch_attn_ring_step": [P, I32, I32, VP, VP, S, I32, VP, VP, VP, VP, VP],
+        "branch_attn_ring_finish": [P, I32, VP, VP, S] + [VP] * 8 + [VP],
         "ba_launch_count": [],
         "ba_last_error": [],
         "ba_version": [],
@@ -370,6 +377,87 @@ def lse_merge(o_a, lse_a, o_b, lse_b, o_out, lse_out, stream=None) -> None:
                          _stream(stream)))
 
 
+# ---- zigzag ring across ranks ------------------------------------------------
+def ba_zigzag_shard(cu_seqlens, branch_anchor, branch_depth, C: int, shard: int) -> dict:
+    """Local problem of one zigzag shard, from host int32 arrays of the whole
+    batch: {"cu_local", "anchor_local", "depth_local", "main_rows",
+    "branch_rows"} as numpy int32 arrays (see the C declaration)."""
+    import numpy as np
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    an = np.ascontiguousarray(branch_anchor, dtype=np.int32)
+    de = np.ascontiguousarray(branch_depth, dtype=np.int32)
+    n_seqs, n_br = cu.shape[0] - 1, an.shape[0]
+    if de.shape[0] != n_br:
+        raise ValueError("branch_anchor and branch_depth differ in length")
+    nm, nb, nbt = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    args = (cu.ctypes.data, n_seqs, an.ctypes.data if n_br else None,
+            de.ctypes.data if n_br else None, n_br, C, shard,
+            ctypes.byref(nm), ctypes.byref(nb), ctypes.byref(nbt))
+    _check(lib.ba_zigzag_shard(*args, None, None, None, None, None))
+    out = {"cu_local": np.zeros(n_seqs + 1, np.int32), "anchor_local": np.zeros(nb.value, np.int32),
+           "depth_local": np.zeros(nb.value, np.int32), "main_rows": np.zeros(nm.value, np.int32),
+           "branch_rows": np.zeros(nbt.value, np.int32)}
+    ptrs = [out[k].ctypes.data if out[k].size else None
+            for k in ("cu_local", "anchor_local", "depth_local", "main_rows", "branch_rows")]
+    _check(lib.ba_zigzag_shard(*args, *ptrs))
+    return out
+
+
+def ba_ring_workspace_size(local: Problem, C: int):
+    """(plan_bytes, acc_bytes) of one ring rank."""
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib.ba_ring_workspace_size(ctypes.byref(local.c), C, ctypes.byref(a),
+                                      ctypes.byref(b)))
+    return a.value, b.value
+
+
+def ba_ring_plan(local: Problem, C: int, shard: int, step: int, cu_global, cu_visit, plan_ws,
+                 stream=None) -> None:
+    import torch
+    _expect_index_arrays(local, "device")
+    _expect(plan_ws, (plan_ws.numel(),), torch.uint8, "plan_ws")
+    for name, t in (("cu_global", cu_global), ("cu_visit", cu_visit)):
+        if step > 0:
+            _expect(t, (local.c.n_seqs + 1,), torch.int32, name)
+    _check(lib.ba_ring_plan(ctypes.byref(local.c), C, shard, step,
+                            _ptr(cu_global) if step > 0 else None,
+                            _ptr(cu_visit) if step > 0 else None, _ptr(plan_ws), plan_ws.numel(),
+                            _stream(stream)))
+
+
+def branch_attn_ring_step(local: Problem, C: int, step: int, plan_ws, acc_ws, q_m, k_m_visit,
+                          v_m_visit, q_b, stream=None) -> None:
+    import torch
+    _expect_ws(plan_ws, "plan_ws")
+    _expect_ws(acc_ws, "acc_ws")
+    sh = local.shapes()
+    _expect(q_m, sh["q_m"], torch.bfloat16, "q_m")
+    _expect(q_b, sh["q_b"], torch.bfloat16, "q_b")
+    n_visit = k_m_visit.shape[0]
+    for name, t in (("k_m_visit", k_m_visit), ("v_m_visit", v_m_visit)):
+        _expect(t, (n_visit, local.c.hkv, local.c.head_dim), torch.bfloat16, name)
+    _check(lib.branch_attn_ring_step(ctypes.byref(local.c), C, step, _ptr(plan_ws), _ptr(acc_ws),
+                                     acc_ws.numel() * acc_ws.element_size(), n_visit, _ptr(q_m),
+                                     _ptr(k_m_visit), _ptr(v_m_visit), _ptr(q_b), _stream(stream)))
+
+
+def branch_attn_ring_finish(local: Problem, C: int, plan_ws, acc_ws, q_m, q_b, k_b, v_b, o_m, o_b,
+                            lse_m, lse_b, stream=None) -> None:
+    import torch
+    _expect_ws(plan_ws, "plan_ws")
+    _expect_ws(acc_ws, "acc_ws")
+    sh = local.shapes()
+    for name, t, like in (("q_m", q_m, "q_m"), ("q_b", q_b, "q_b"), ("k_b", k_b, "k_b"),
+                          ("v_b", v_b, "v_b"), ("o_m", o_m, "q_m"), ("o_b", o_b, "q_b")):
+        _expect(t, sh[like], torch.bfloat16, name)
+    _expect(lse_m, sh["lse_m"], torch.float32, "lse_m")
+    _expect(lse_b, sh["lse_b"], torch.float32, "lse_b")
+    _check(lib.branch_attn_ring_finish(
+        ctypes.byref(local.c), C, _ptr(plan_ws), _ptr(acc_ws),
+        acc_ws.numel() * acc_ws.element_size(), _ptr(q_m), _ptr(q_b), _ptr(k_b), _ptr(v_b),
+        _ptr(o_m), _ptr(o_b), _ptr(lse_m), _ptr(lse_b), _stream(stream)))
+
+
 def ba_set_kernel_family(family: int) -> None:
     _check(lib.ba_set_kernel_family(family))
 
@@ -411,3 +499,5 @@ def ba_version() -> str:
 
 
 from .runner import BranchAttention  # noqa: E402,F401
+from . import ring  # noqa: E402,F401
+from .ring import RingSchedule, ZigzagRingAttention  # noqa: E402,F401

@@ -194,6 +194,8 @@ AttnParams make_params(const ba_problem &p, const ba_plan_layout &L, const void 
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.zz_step = -1;
   a.zz_C = p.zigzag_C;
+  a.ring = 0;
+  a.n_keys_m = p.n_main;
   return a;
 }
 
@@ -392,6 +394,226 @@ ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws, void *bwd_ws
   if (fused) BA_TRY(launch_dq_convert(a, (__nv_bfloat16 *)dq_m, (__nv_bfloat16 *)dq_b, s));
   record_event(1, false, s);
   return BA_OK;
+}
+
+// ---- zigzag ring across ranks ---------------------------------------------
+
+ba_status ba_zigzag_shard(const int32_t *cu, int32_t n_seqs, const int32_t *anchor,
+                          const int32_t *depth, int32_t n_branches, int32_t C, int32_t shard,
+                          int32_t *n_main_local, int32_t *n_branches_local,
+                          int32_t *n_branch_tokens_local, int32_t *cu_local,
+                          int32_t *anchor_local, int32_t *depth_local, int32_t *main_rows,
+                          int32_t *branch_rows) {
+  if (!cu || n_seqs < 1 || n_branches < 0 || (n_branches > 0 && (!anchor || !depth))) {
+    set_error("ba_zigzag_shard: cu_seqlens, anchors and depths are required (host arrays)");
+    return BA_ERR_INVALID_ARG;
+  }
+  if (C < 1 || C > 64 || shard < 0 || shard >= C) {
+    set_error("ba_zigzag_shard: need 1 <= C <= 64 and 0 <= shard < C (C %d, shard %d)", C, shard);
+    return BA_ERR_INVALID_ARG;
+  }
+  if (!n_main_local || !n_branches_local || !n_branch_tokens_local) {
+    set_error("ba_zigzag_shard: the three count pointers are required");
+    return BA_ERR_INVALID_ARG;
+  }
+  if (cu[0] != 0) {
+    set_error("ba_zigzag_shard: cu_seqlens[0] must be 0");
+    return BA_ERR_INVALID_ARG;
+  }
+  for (int s = 0; s < n_seqs; ++s) {
+    const int64_t L = (int64_t)cu[s + 1] - cu[s];
+    if (L < 2 * C) {
+      set_error("ba_zigzag_shard: sequence %d holds %lld tokens, fewer than 2C = %d", s,
+                (long long)L, 2 * C);
+      return L < 1 ? BA_ERR_INVALID_ARG : BA_ERR_UNSUPPORTED;
+    }
+  }
+  // chunk k of sequence s: [cu[s] + floor(kL/2C), cu[s] + floor((k+1)L/2C))
+  auto chunk = [&](int s, int k, int64_t *a, int64_t *b) {
+    const int64_t L = (int64_t)cu[s + 1] - cu[s];
+    *a = cu[s] + (k * L) / (2 * C);
+    *b = cu[s] + ((k + 1) * L) / (2 * C);
+  };
+  int64_t nm = 0, nb = 0, nbt = 0;
+  if (cu_local) cu_local[0] = 0;
+  int b = 0;          // branches are sorted by anchor
+  int64_t brow = 0;   // first branch row of branch b
+  for (int s = 0; s < n_seqs; ++s) {
+    for (int piece = 0; piece < 2; ++piece) {
+      int64_t a0, a1;
+      chunk(s, piece == 0 ? shard : 2 * C - 1 - shard, &a0, &a1);
+      // main rows a0..a1-1 become local rows nm .. nm + (a1 - a0) - 1
+      while (b < n_branches && anchor[b] < a0) brow += depth[b++];
+      int bb = b;
+      int64_t bbrow = brow;
+      while (bb < n_branches && anchor[bb] < a1) {
+        if (anchor[bb] < a0) {  // anchors must be sorted
+          set_error("ba_zigzag_shard: branch anchors must be non-decreasing");
+          return BA_ERR_INVALID_ARG;
+        }
+        if (anchor_local) anchor_local[nb] = (int32_t)(nm + (anchor[bb] - a0));
+        if (depth_local) depth_local[nb] = depth[bb];
+        for (int j = 0; j < depth[bb]; ++j)
+          if (branch_rows) branch_rows[nbt + j] = (int32_t)(bbrow + j);
+        nbt += depth[bb];
+        bbrow += depth[bb];
+        ++nb;
+        ++bb;
+      }
+      if (main_rows)
+        for (int64_t r = a0; r < a1; ++r) main_rows[nm + (r - a0)] = (int32_t)r;
+      nm += a1 - a0;
+    }
+    if (cu_local) cu_local[s + 1] = (int32_t)nm;
+  }
+  *n_main_local = (int32_t)nm;
+  *n_branches_local = (int32_t)nb;
+  *n_branch_tokens_local = (int32_t)nbt;
+  return BA_OK;
+}
+
+ba_status ba_ring_workspace_size(const ba_problem *local, int32_t C, size_t *plan_bytes,
+                                 size_t *acc_bytes) {
+  BA_TRY(validate_problem(local, false));
+  if (C < 1 || C > 64) {
+    set_error("ring size C must be in [1, 64] (got %d)", C);
+    return BA_ERR_INVALID_ARG;
+  }
+  ba_plan_layout L;
+  plan_layout(*local, &L);
+  const size_t rows = (size_t)local->n_main + local->n_branch_tokens;
+  if (plan_bytes) *plan_bytes = L.total_bytes;
+  if (acc_bytes)
+    *acc_bytes = align_up(4 * rows * local->hq * local->head_dim, 256) +
+                 align_up(4 * rows * local->hq, 256);
+  return BA_OK;
+}
+
+namespace {
+ba_status check_ring(const ba_problem *local, int32_t C, int32_t step, bool allow_last) {
+  BA_TRY(validate_problem(local, true));
+  if (local->zigzag_C != 1) {
+    set_error("the shard-local problem must have zigzag_C = 1 (the ring size is passed apart)");
+    return BA_ERR_INVALID_ARG;
+  }
+  if (C < 1 || C > 64 || step < 0 || step > (allow_last ? C : C - 1)) {
+    set_error("ring: need 1 <= C <= 64 and 0 <= step < C (C %d, step %d)", C, step);
+    return BA_ERR_INVALID_ARG;
+  }
+  return BA_OK;
+}
+
+ba_status ring_acc(const ba_problem *local, int32_t C, void *acc_ws, size_t acc_bytes,
+                   AttnParams *a) {
+  size_t need = 0;
+  BA_TRY(ba_ring_workspace_size(local, C, nullptr, &need));
+  BA_TRY(check_tensor(acc_ws, true, "acc_ws"));
+  if (acc_bytes < need) {
+    set_error("ring accumulator too small: %zu < %zu bytes", acc_bytes, need);
+    return BA_ERR_WORKSPACE_TOO_SMALL;
+  }
+  const size_t rows = (size_t)local->n_main + local->n_branch_tokens;
+  a->zz_o = reinterpret_cast<float *>(acc_ws);
+  a->zz_lse = reinterpret_cast<float *>(reinterpret_cast<char *>(acc_ws) +
+                                        align_up(4 * rows * local->hq * local->head_dim, 256));
+  return BA_OK;
+}
+}  // namespace
+
+ba_status ba_ring_plan(const ba_problem *local, int32_t C, int32_t shard, int32_t step,
+                       const int32_t *cu_global, const int32_t *cu_visit, void *plan_ws,
+                       size_t plan_bytes, ba_stream_t stream) {
+  BA_TRY(check_ring(local, C, step, false));
+  if (shard < 0 || shard >= C) {
+    set_error("ring: shard %d outside [0, %d)", shard, C);
+    return BA_ERR_INVALID_ARG;
+  }
+  BA_TRY(check_plan_ws(plan_ws));
+  ba_plan_layout L;
+  plan_layout(*local, &L);
+  if (plan_bytes < L.total_bytes) {
+    set_error("plan workspace too small: %zu < %zu bytes", plan_bytes, L.total_bytes);
+    return BA_ERR_WORKSPACE_TOO_SMALL;
+  }
+  if (step == 0) return launch_plan(*local, L, plan_view(L, plan_ws), (cudaStream_t)stream);
+  if (!cu_global || !cu_visit || !aligned(cu_global, 4) || !aligned(cu_visit, 4)) {
+    set_error("ring plan: cu_global and cu_visit must be 4-byte aligned device arrays");
+    return cu_global && cu_visit ? BA_ERR_MISALIGNED : BA_ERR_INVALID_ARG;
+  }
+  const int j = ((shard - step) % C + C) % C;
+  return launch_ring_plan(*local, L, plan_view(L, plan_ws), cu_global, cu_visit, C, shard, j,
+                          (cudaStream_t)stream);
+}
+
+ba_status branch_attn_ring_step(const ba_problem *local, int32_t C, int32_t step,
+                                const void *plan_ws, void *acc_ws, size_t acc_bytes,
+                                int32_t n_main_visit, const void *q_m, const void *k_m_visit,
+                                const void *v_m_visit, const void *q_b, ba_stream_t stream) {
+  BA_TRY(check_ring(local, C, step, false));
+  BA_TRY(check_plan_ws(plan_ws));
+  if (n_main_visit < 1 || n_main_visit > kMaxRows) {
+    set_error("n_main_visit must be in [1, 2^28] (got %d)", n_main_visit);
+    return BA_ERR_INVALID_ARG;
+  }
+  const bool br = local->n_branch_tokens > 0;
+  BA_TRY(check_tensor(q_m, true, "q_m"));
+  BA_TRY(check_tensor(k_m_visit, true, "k_m_visit"));
+  BA_TRY(check_tensor(v_m_visit, true, "v_m_visit"));
+  BA_TRY(check_tensor(q_b, br, "q_b"));
+  ba_plan_layout L;
+  plan_layout(*local, &L);
+  AttnParams a = make_params(*local, L, plan_ws);
+  BA_TRY(ring_acc(local, C, acc_ws, acc_bytes, &a));
+  a.ring = 1;
+  a.zz_step = step;
+  a.zz_C = C;
+  a.n_keys_m = n_main_visit;
+  a.q_m = (const __nv_bfloat16 *)q_m;
+  a.k_m = (const __nv_bfloat16 *)k_m_visit;
+  a.v_m = (const __nv_bfloat16 *)v_m_visit;
+  a.q_b = (const __nv_bfloat16 *)q_b;
+  cudaStream_t s = (cudaStream_t)stream;
+  record_event(0, true, s);
+  ba_status st = launch_fwd_sm100(a, s);
+  record_event(0, false, s);
+  return st;
+}
+
+ba_status branch_attn_ring_finish(const ba_problem *local, int32_t C, const void *plan_ws,
+                                  void *acc_ws, size_t acc_bytes, const void *q_m,
+                                  const void *q_b, const void *k_b, const void *v_b, void *o_m,
+                                  void *o_b, float *lse_m, float *lse_b, ba_stream_t stream) {
+  BA_TRY(check_ring(local, C, C, true));
+  BA_TRY(check_plan_ws(plan_ws));
+  const bool br = local->n_branch_tokens > 0;
+  BA_TRY(check_tensor(q_m, true, "q_m"));
+  BA_TRY(check_tensor(o_m, true, "o_m"));
+  BA_TRY(check_tensor(q_b, br, "q_b"));
+  BA_TRY(check_tensor(k_b, br, "k_b"));
+  BA_TRY(check_tensor(v_b, br, "v_b"));
+  BA_TRY(check_tensor(o_b, br, "o_b"));
+  BA_TRY(check_f32(lse_m, true, "lse_m"));
+  BA_TRY(check_f32(lse_b, br, "lse_b"));
+  ba_plan_layout L;
+  plan_layout(*local, &L);
+  AttnParams a = make_params(*local, L, plan_ws);
+  BA_TRY(ring_acc(local, C, acc_ws, acc_bytes, &a));
+  a.ring = 1;
+  a.zz_step = C;
+  a.zz_C = C;
+  a.q_m = (const __nv_bfloat16 *)q_m;
+  a.q_b = (const __nv_bfloat16 *)q_b;
+  a.k_b = (const __nv_bfloat16 *)k_b;
+  a.v_b = (const __nv_bfloat16 *)v_b;
+  a.o_m = (__nv_bfloat16 *)o_m;
+  a.o_b = (__nv_bfloat16 *)o_b;
+  a.lse_m = lse_m;
+  a.lse_b = lse_b;
+  cudaStream_t s = (cudaStream_t)stream;
+  record_event(0, true, s);
+  ba_status st = launch_fwd_sm100(a, s);
+  record_event(0, false, s);
+  return st;
 }
 
 ba_status lse_merge(int64_t rows, int32_t heads, int32_t head_dim, int32_t o_is_fp32,

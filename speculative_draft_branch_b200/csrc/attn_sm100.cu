@@ -250,11 +250,15 @@ __global__ void __launch_bounds__(256, 1)
     const int zz = a.zz_step;
     if (valid) {
       const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[row_off + row0 + row];
-      if (zz < 0 || zz == a.zz_C) {
+      if (a.ring) {
+        // ring mode: this step's main interval, or the branch-local one last
+        if (zz < a.zz_C) { lo[0] = iv.x; hi[0] = iv.y; }
+        else { lo[2] = iv.z; hi[2] = iv.w; }
+      } else if (zz < 0 || zz == a.zz_C) {
         lo[0] = iv.x; hi[0] = iv.y;
         lo[2] = iv.z; hi[2] = iv.w;
       }
-      if (zz >= 0 && zz < a.zz_C) {
+      if (!a.ring && zz >= 0 && zz < a.zz_C) {
         int s_lo = 0, s_hi = a.n_seqs;
         while (s_lo < s_hi) {
           const int mid = (s_lo + s_hi + 1) >> 1;
@@ -630,11 +634,15 @@ __global__ void __launch_bounds__(384, 1)
     const int zz = a.zz_step;
     if (valid) {
       const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[row_off + row0 + row];
-      if (zz < 0 || zz == a.zz_C) {
+      if (a.ring) {
+        // ring mode: this step's main interval, or the branch-local one last
+        if (zz < a.zz_C) { lo[0] = iv.x; hi[0] = iv.y; }
+        else { lo[2] = iv.z; hi[2] = iv.w; }
+      } else if (zz < 0 || zz == a.zz_C) {
         lo[0] = iv.x; hi[0] = iv.y;
         lo[2] = iv.z; hi[2] = iv.w;
       }
-      if (zz >= 0 && zz < a.zz_C) {
+      if (!a.ring && zz >= 0 && zz < a.zz_C) {
         int s_lo = 0, s_hi = a.n_seqs;
         while (s_lo < s_hi) {
           const int mid = (s_lo + s_hi + 1) >> 1;
@@ -829,21 +837,30 @@ ba_status launch_exp2_check(const float *x, float *y_fma, float *y_mufu, int64_t
 
 
 ba_status launch_fwd_sm100(const AttnParams &a, cudaStream_t s) {
-  TensorMaps tm;
+  TensorMaps tm = {};
   const int d = a.head_dim;
   ba_status st;
+  // a ring step reads only the visiting shard's main K/V; the ring's last
+  // step only the local branch K/V; maps that a launch never reads alias one
+  // that it does
+  const bool need_main_kv = !(a.ring && a.zz_step == a.zz_C);
+  const bool need_branch_kv = a.n_bt > 0 && !(a.ring && a.zz_step < a.zz_C);
   if ((st = make_tensor_map(&tm.q_m, a.q_m, a.n_main, a.hq, d, 128)) != BA_OK) return st;
-  if ((st = make_tensor_map(&tm.k_m, a.k_m, a.n_main, a.hkv, d, 128)) != BA_OK) return st;
-  if ((st = make_tensor_map(&tm.v_m, a.v_m, a.n_main, a.hkv, d, 128)) != BA_OK) return st;
   if (a.n_bt > 0) {
     if ((st = make_tensor_map(&tm.q_b, a.q_b, a.n_bt, a.hq, d, 128)) != BA_OK) return st;
-    if ((st = make_tensor_map(&tm.k_b, a.k_b, a.n_bt, a.hkv, d, 128)) != BA_OK) return st;
-    if ((st = make_tensor_map(&tm.v_b, a.v_b, a.n_bt, a.hkv, d, 128)) != BA_OK) return st;
   } else {
     tm.q_b = tm.q_m;
-    tm.k_b = tm.k_m;
-    tm.v_b = tm.v_m;
   }
+  if (need_main_kv) {
+    if ((st = make_tensor_map(&tm.k_m, a.k_m, a.n_keys_m, a.hkv, d, 128)) != BA_OK) return st;
+    if ((st = make_tensor_map(&tm.v_m, a.v_m, a.n_keys_m, a.hkv, d, 128)) != BA_OK) return st;
+  }
+  if (need_branch_kv) {
+    if ((st = make_tensor_map(&tm.k_b, a.k_b, a.n_bt, a.hkv, d, 128)) != BA_OK) return st;
+    if ((st = make_tensor_map(&tm.v_b, a.v_b, a.n_bt, a.hkv, d, 128)) != BA_OK) return st;
+  }
+  if (!need_main_kv) { tm.k_m = tm.k_b; tm.v_m = tm.v_b; }
+  if (!need_branch_kv) { tm.k_b = tm.k_m; tm.v_b = tm.v_m; }
   const int64_t grid = (int64_t)a.n_qt * a.hq;
   if (grid == 0) return BA_OK;
   cudaError_t e;

@@ -50,13 +50,13 @@ __device__ __forceinline__ TileSegs make_segs(const AttnParams &a, int t, bool i
   int n = 0;
   const int32_t *qt = a.plan.qtile + (int64_t)t * 6;
   const int zz = a.zz_step;
-  if (zz < 0) {
-    const int k0 = qt[0] * 128, k1 = min(qt[3] * 128, a.n_main);
-    ts.s[n++] = {k0, (k1 - k0 + 127) / 128, 0, qt[1] * 128, qt[2] * 128};
+  if (zz < 0 || (a.ring && zz < a.zz_C)) {
+    const int k0 = qt[0] * 128, k1 = min(qt[3] * 128, a.n_keys_m);
+    if (k1 > k0) ts.s[n++] = {k0, (k1 - k0 + 127) / 128, 0, qt[1] * 128, qt[2] * 128};
   } else if (zz < a.zz_C) {
     const int32_t *z = a.plan.zz_tiles + ((int64_t)zz * a.n_qt + t) * 4;
     for (int w = 0; w < 2; ++w) {
-      const int k0 = z[2 * w] * 128, k1 = min(z[2 * w + 1] * 128, a.n_main);
+      const int k0 = z[2 * w] * 128, k1 = min(z[2 * w + 1] * 128, a.n_keys_m);
       if (k1 > k0) ts.s[n++] = {k0, (k1 - k0 + 127) / 128, w, 0, 0};
     }
   }

@@ -51,6 +51,11 @@ struct AttnParams {
   float *zz_lse;
   int32_t zz_step;            // ring step, -1 = monolithic, C = branch-local pass
   int32_t zz_C;
+  // ring mode (zigzag context parallelism across ranks): the plan holds this
+  // step's main-key intervals in row_iv (x, y) and tile ranges in qtile[0..3];
+  // step C takes the branch-local keys (row_iv z, w; qtile[4..5])
+  int32_t ring;
+  int32_t n_keys_m;           // main key rows (the visiting shard's in ring mode, else n_main)
   const int32_t *cu_seqlens;
   PlanView plan;
   int32_t n_main, n_bt;       // main / branch token counts
@@ -69,6 +74,9 @@ ba_status cuda_check(cudaError_t e, const char *what);
 
 ba_status launch_plan(const ba_problem &p, const ba_plan_layout &L, const PlanView &v,
                       cudaStream_t s);
+ba_status launch_ring_plan(const ba_problem &p, const ba_plan_layout &L, const PlanView &v,
+                           const int32_t *cu_glob, const int32_t *cu_vis, int C, int q, int j,
+                           cudaStream_t s);
 ba_status launch_lse_merge(int64_t rows, int heads, int d, int fp32, const void *oa,
                            const float *la, const void *ob, const float *lb, void *oo,
                            float *lo, cudaStream_t s);

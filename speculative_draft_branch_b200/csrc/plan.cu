@@ -272,7 +272,113 @@ __global__ void plan_zz_kernel(const int32_t *cu, int n_seqs, int C, int n_main,
   o[3] = hi1 >= 0 ? hi1 / kTileN + 1 : 0;
 }
 
+// ---- ring steps (zigzag context parallelism across ranks) -----------------
+// A rank holding shard q keeps chunks q and 2C-1-q of every sequence (chunk k
+// of a sequence of length L covers positions [floor(kL/2C), floor((k+1)L/2C)))
+// as one packed problem, in position order.  Against the main keys of another
+// shard j (held in the same shard-local order by the rank it came from), a
+// chunk of keys is either wholly before a query's position or wholly after it:
+//   j < q: every query of the sequence sees shard j's first chunk (chunk j);
+//   j > q: queries in the second chunk (2C-1-q) see all of shard j's keys of
+//          the sequence, queries in the first chunk none.
+// A branch query takes its anchor's chunk (the anchor is a main position).
+// Step 0 (j = q) is the causal plan of the shard-local problem itself.
+__device__ __forceinline__ int chunk_len(int64_t L, int C, int k) {
+  return (int)(((k + 1) * L) / (2 * C) - (k * L) / (2 * C));
+}
+
+__device__ __forceinline__ int2 ring_interval(const int32_t *cu_loc, const int32_t *cu_glob,
+                                              const int32_t *cu_vis, int n_seqs, int C, int q,
+                                              int j, int local_row) {
+  const int s = upper_index(cu_loc, n_seqs + 1, local_row);
+  const int pos = local_row - cu_loc[s];
+  const int64_t L = cu_glob[s + 1] - cu_glob[s];
+  const bool second = pos >= chunk_len(L, C, q);
+  const int lo = cu_vis[s];
+  int hi;
+  if (j < q) hi = lo + chunk_len(L, C, j) - 1;
+  else hi = second ? cu_vis[s + 1] - 1 : lo - 1;
+  return make_int2(lo, hi);
+}
+
+__global__ void plan_ring_rows_kernel(const int32_t *cu_loc, const int32_t *cu_glob,
+                                      const int32_t *cu_vis, const int32_t *anchor, int n_seqs,
+                                      int n_main, int n_br, int C, int q, int j,
+                                      const int32_t *status, const int32_t *cu_branch,
+                                      int32_t *row_iv) {
+  if (status[0] != 0) return;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n_main) {
+    const int2 v = ring_interval(cu_loc, cu_glob, cu_vis, n_seqs, C, q, j, (int)i);
+    reinterpret_cast<int4 *>(row_iv)[i] = make_int4(v.x, v.y, 0, -1);
+  }
+  if (i < n_br) {
+    const int b = (int)i;
+    const int2 v = ring_interval(cu_loc, cu_glob, cu_vis, n_seqs, C, q, j, anchor[b]);
+    for (int r = cu_branch[b]; r < cu_branch[b + 1]; ++r)
+      reinterpret_cast<int4 *>(row_iv)[n_main + r] = make_int4(v.x, v.y, 0, -1);
+  }
+}
+
+// Per query tile: the key tiles any row sees, and those every row sees whole.
+__global__ void plan_ring_tiles_kernel(int n_main, int n_bt, int n_qt_main, int n_qt,
+                                       const int32_t *status, const int32_t *row_iv,
+                                       int32_t *qtile, int32_t *fwd_cost) {
+  if (status[0] != 0) return;
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n_qt) return;
+  const bool is_main = t < n_qt_main;
+  const int tt = is_main ? t : t - n_qt_main;
+  const int rows = is_main ? n_main : n_bt;
+  const int off = is_main ? 0 : n_main;
+  const int r0 = tt * kTileM, r1 = min(r0 + kTileM, rows);
+  int lo_min = INT32_MAX, hi_max = -1, lo_max = -1, hi_min = INT32_MAX;
+  bool every = r1 - r0 == kTileM;
+  for (int r = r0; r < r1; ++r) {
+    const int4 iv = reinterpret_cast<const int4 *>(row_iv)[off + r];
+    if (iv.y >= iv.x) {
+      lo_min = min(lo_min, iv.x); hi_max = max(hi_max, iv.y);
+      lo_max = max(lo_max, iv.x); hi_min = min(hi_min, iv.y);
+    } else {
+      every = false;
+    }
+  }
+  int kb = 0, ke = 0, fb = 0, fe = 0;
+  if (hi_max >= 0) {
+    kb = lo_min / kTileN;
+    ke = hi_max / kTileN + 1;
+    fb = (lo_max + kTileN - 1) / kTileN;
+    fe = (hi_min + 1) / kTileN;
+    if (!every || fb >= fe) { fb = kb; fe = kb; }
+  }
+  int32_t *o = qtile + (int64_t)t * 6;
+  o[0] = kb; o[1] = fb; o[2] = fe; o[3] = ke; o[4] = 0; o[5] = 0;
+  fwd_cost[t] = ke - kb;
+}
+
 }  // namespace
+
+ba_status launch_ring_plan(const ba_problem &p, const ba_plan_layout &L, const PlanView &v,
+                           const int32_t *cu_glob, const int32_t *cu_vis, int C, int q, int j,
+                           cudaStream_t s) {
+  const int n_qt = L.n_qtiles_main + L.n_qtiles_branch;
+  plan_scan_kernel<<<1, kScanThreads, 0, s>>>(p.cu_seqlens, p.branch_anchor, p.branch_depth,
+                                              p.n_seqs, p.n_main, p.n_branches,
+                                              p.n_branch_tokens, v.status, v.cu_branch);
+  ba_status st = cuda_check(cudaGetLastError(), "plan_scan_kernel launch");
+  if (st != BA_OK) return st;
+  const int64_t nrow = p.n_main > p.n_branches ? p.n_main : p.n_branches;
+  plan_ring_rows_kernel<<<(unsigned)cdiv64(nrow, 256), 256, 0, s>>>(
+      p.cu_seqlens, cu_glob, cu_vis, p.branch_anchor, p.n_seqs, p.n_main, p.n_branches, C, q, j,
+      v.status, v.cu_branch, v.row_iv);
+  plan_ring_tiles_kernel<<<(unsigned)cdiv64(n_qt, 128), 128, 0, s>>>(
+      p.n_main, p.n_branch_tokens, L.n_qtiles_main, n_qt, v.status, v.row_iv, v.qtile,
+      v.fwd_cost);
+  plan_rank_kernel<<<(unsigned)cdiv64(n_qt, kRankThreads), kRankThreads, 0, s>>>(
+      v.status, v.fwd_cost, n_qt, v.fwd_order);
+  count_launches(4);
+  return cuda_check(cudaGetLastError(), "ring plan kernels launch");
+}
 
 ba_status launch_plan(const ba_problem &p, const ba_plan_layout &L, const PlanView &v,
                       cudaStream_t s) {
