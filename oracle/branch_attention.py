@@ -425,10 +425,11 @@ def keys_backward(st, t, main_keys=(), branch_keys=(), groups=None, operand_bf16
     [len(branch_keys), Hkv, d]; only kv heads in `groups` (default: all) are
     computed, each summed over all q heads of its group.
 
-    operand_bf16=True rounds P and dS to bf16 before they multiply dO and q
-    (everything else stays fp64): the precision in which a bf16 tensor-core
-    product receives them, so that a kernel's error can be separated from what
-    the rounding of those operands alone causes.
+    operand_bf16=True rounds P and dS to bf16 before they multiply dO and q,
+    and takes D = dO . O from the bf16-rounded O (everything else stays fp64):
+    the precision in which a bf16 tensor-core backward receives them (its O is
+    the forward's bf16 output), so that a kernel's error can be separated from
+    what the rounding of those operands alone causes.
     """
     return _keys_backward(st, t, main_keys, branch_keys, groups, (bool(operand_bf16),))[0]
 
@@ -485,14 +486,18 @@ def _keys_backward(st, t, main_keys, branch_keys, groups, modes):
            for _ in modes]
     for h in heads:
         g = h // grp
-        dd = (dox[:, h] * fw["o"][:, h]).sum(axis=1)                # D_i = dO_i . O_i
+        # D_i = dO_i . O_i; with bf16 operands O is the forward's bf16 output
+        dd = {False: (dox[:, h] * fw["o"][:, h]).sum(axis=1)}
+        if True in modes:
+            dd[True] = (dox[:, h] * round_bf16(fw["o"][:, h])).sum(axis=1)
         for vis, ksel, vsel, kind in ((vis_m, km_sel, vm_sel, "m"), (vis_b, kb_sel, vb_sel, "b")):
             if ksel.shape[0] == 0:
                 continue
             s_ik = st.scale * (qx[:, h] @ ksel[:, g].T)             # [R, keys]
             p = np.where(vis, np.exp(np.where(vis, s_ik, 0.0) - fw["lse"][h][:, None]), 0.0)
-            ds = p * (dox[:, h] @ vsel[:, g].T - dd[:, None])
+            dp = dox[:, h] @ vsel[:, g].T
             for out, rounded in zip(res, modes):
+                ds = p * (dp - dd[rounded][:, None])
                 pp, dss = (round_bf16(p), round_bf16(ds)) if rounded else (p, ds)
                 out["dv_" + kind][:, g] += pp.T @ dox[:, h]
                 out["dk_" + kind][:, g] += st.scale * (dss.T @ qx[:, h])

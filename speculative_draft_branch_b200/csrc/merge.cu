@@ -1,7 +1,9 @@
 // Streaming (HBM-bound) kernels: the standalone online-softmax merge, the
 // backward preprocess D = rowsum(dO * O), and the dQ fp32 -> bf16 convert.
-// All use 16-byte vector accesses, one row-head per group of lanes, and a
-// grid of (SM count x resident blocks) that strides over the row-heads.
+// All use 16-byte vector accesses and a grid of (SM count x resident blocks)
+// that strides over the work: the merge and the convert take one row-head
+// per group of lanes, the preprocess one row per lane (32 rows of one head
+// per warp, so that its per-head outputs are written in contiguous runs).
 #include "internal.cuh"
 
 namespace ba {
@@ -96,74 +98,72 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, int heads,
 
 // ---- backward preprocess ---------------------------------------------------
 // D[h, row] = sum_d dO[row, h, d] * O[row, h, d] (fp32 accumulate), rows =
-// main rows then branch rows; when the backward accumulates dQ with atomics
-// the fp32 dQ accumulator of the same row-head is zeroed in the same pass.
+// main rows then branch rows, and the per-query records the backward reads
+// {l log2 e, D, key lo, key hi} (main-key interval and branch-local interval).
+// A warp takes 32 consecutive rows of one head, one lane per row: each lane
+// streams its row's 2 d bf16 of O and dO (16-byte loads, all issued before
+// the products), and the warp's writes of D and of the records are 128- and
+// 512-byte contiguous runs.  When the backward accumulates dQ in fp32 the
+// accumulator of the same row-head is zeroed in the same pass.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(AttnParams a) {
-  constexpr int kLanes = D / 8;
-  constexpr int kPerWarp = 32 / kLanes;
-  const int lane = threadIdx.x % kLanes;
-  const int64_t rows = (int64_t)a.n_main + a.n_bt;
-  const int64_t total = rows * a.hq;
+  constexpr int kVec = D / 8;  // 16-byte vectors per row-head
   if (a.plan.status[0] != 0) return;
+  const int64_t rows = (int64_t)a.n_main + a.n_bt;
+  const int64_t blocks32 = (rows + 31) / 32;
+  const int64_t tasks = blocks32 * a.hq;
+  const int lane = threadIdx.x % 32;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
-  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-       w * kPerWarp < total; w += warps) {
-    const int64_t g = w * kPerWarp + (threadIdx.x % 32) / kLanes;
-    const bool active = g < total;
+  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; w < tasks;
+       w += warps) {
+    const int h = (int)(w % a.hq);
+    const int64_t row = (w / a.hq) * 32 + lane;
+    if (row >= rows) continue;
+    const bool is_main = row < a.n_main;
+    const int64_t r = is_main ? row : row - a.n_main;
+    const int64_t off = (r * a.hq + h) * D;
+    const uint4 *o4 = reinterpret_cast<const uint4 *>((is_main ? a.o_m : a.o_b) + off);
+    const uint4 *d4 = reinterpret_cast<const uint4 *>((is_main ? a.do_m : a.do_b) + off);
+    uint4 ov[kVec], dv[kVec];
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      ov[i] = o4[i];
+      dv[i] = d4[i];
+    }
     float s = 0.f;
-    int64_t row = 0;
-    int h = 0;
-    if (active) {
-      row = g / a.hq;
-      h = (int)(g % a.hq);
-      const bool is_main = row < a.n_main;
-      const int64_t r = is_main ? row : row - a.n_main;
-      const __nv_bfloat16 *o = is_main ? a.o_m : a.o_b;
-      const __nv_bfloat16 *dout = is_main ? a.do_m : a.do_b;
-      const int64_t off = (r * a.hq + h) * D + lane * 8;
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
       float x[8], y[8];
-      unpack8(*reinterpret_cast<const uint4 *>(o + off), x);
-      unpack8(*reinterpret_cast<const uint4 *>(dout + off), y);
+      unpack8(ov[i], x);
+      unpack8(dv[i], y);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) s += x[i] * y[i];
-      if (a.zero_dq_acc) {
-        float4 *dq = reinterpret_cast<float4 *>(a.dq_acc + (row * a.hq + h) * D + lane * 8);
-        dq[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        dq[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      for (int e = 0; e < 8; ++e) s = fmaf(x[e], y[e], s);
     }
+    if (a.zero_dq_acc) {
+      float4 *dq = reinterpret_cast<float4 *>(a.dq_acc + (row * a.hq + h) * D);
 #pragma unroll
-    for (int o2 = kLanes / 2; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
-    if (active && lane == 0) {
-      const_cast<float *>(a.d_all)[(int64_t)h * rows + row] = s;
-      if (a.rec) {
-        const bool is_main = row < a.n_main;
-        const int64_t r = is_main ? row : row - a.n_main;
-        const float l2 = (is_main ? a.lse_m : a.lse_b)[(int64_t)h * (is_main ? a.n_main : a.n_bt) + r] *
-                         1.4426950408889634f;
-        const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[row];
-        const int64_t pr = (is_main ? 0 : a.n_main_pad) + r;
-        a.rec[(int64_t)h * a.rows_pad + pr] =
-            make_float4(l2, s, __int_as_float(iv.x), __int_as_float(iv.y));
-        a.rec[((int64_t)a.hq + h) * a.rows_pad + pr] =
-            make_float4(l2, s, __int_as_float(iv.z), __int_as_float(iv.w));
-      }
+      for (int i = 0; i < D / 4; ++i) dq[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    const_cast<float *>(a.d_all)[(int64_t)h * rows + row] = s;
+    const float l2 = (is_main ? a.lse_m : a.lse_b)[(int64_t)h * (is_main ? a.n_main : a.n_bt) + r] *
+                     1.4426950408889634f;
+    const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[row];
+    const int64_t pr = (is_main ? 0 : a.n_main_pad) + r;
+    a.rec[(int64_t)h * a.rows_pad + pr] = make_float4(l2, s, __int_as_float(iv.x), __int_as_float(iv.y));
+    a.rec[((int64_t)a.hq + h) * a.rows_pad + pr] =
+        make_float4(l2, s, __int_as_float(iv.z), __int_as_float(iv.w));
   }
   // padding rows of the records: empty key intervals
-  if (a.rec) {
-    const int pad_m = a.n_main_pad - a.n_main;
-    const int pad_b = a.rows_pad - a.n_main_pad - a.n_bt;
-    const int64_t n_pad = (int64_t)(pad_m + pad_b) * a.hq * 2;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_pad;
-         i += (int64_t)gridDim.x * blockDim.x) {
-      const int per = pad_m + pad_b;
-      const int64_t kh = i / per;
-      const int j = (int)(i % per);
-      const int64_t pr = j < pad_m ? a.n_main + j : a.n_main_pad + a.n_bt + (j - pad_m);
-      a.rec[kh * a.rows_pad + pr] = make_float4(0.f, 0.f, __int_as_float(1), __int_as_float(0));
-    }
+  const int pad_m = a.n_main_pad - a.n_main;
+  const int pad_b = a.rows_pad - a.n_main_pad - a.n_bt;
+  const int64_t n_pad = (int64_t)(pad_m + pad_b) * a.hq * 2;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_pad;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int per = pad_m + pad_b;
+    const int64_t kh = i / per;
+    const int j = (int)(i % per);
+    const int64_t pr = j < pad_m ? a.n_main + j : a.n_main_pad + a.n_bt + (j - pad_m);
+    a.rec[kh * a.rows_pad + pr] = make_float4(0.f, 0.f, __int_as_float(1), __int_as_float(0));
   }
 }
 
@@ -211,11 +211,12 @@ ba_status launch_lse_merge(int64_t rows, int heads, int d, int fp32, const void 
 }
 
 ba_status launch_bwd_preprocess(const AttnParams &a, cudaStream_t s) {
-  const int64_t groups = ((int64_t)a.n_main + a.n_bt) * a.hq;
+  // one warp task per 32 rows of one head; 8 warps per block
+  const int64_t tasks = (((int64_t)a.n_main + a.n_bt + 31) / 32) * a.hq;
   if (a.head_dim == 64)
-    bwd_preprocess_kernel<64><<<grid_for(groups, 256 / 8), 256, 0, s>>>(a);
+    bwd_preprocess_kernel<64><<<grid_for(tasks, 8), 256, 0, s>>>(a);
   else
-    bwd_preprocess_kernel<128><<<grid_for(groups, 256 / 16), 256, 0, s>>>(a);
+    bwd_preprocess_kernel<128><<<grid_for(tasks, 8), 256, 0, s>>>(a);
   count_launches(1);
   return cuda_check(cudaGetLastError(), "bwd_preprocess launch");
 }

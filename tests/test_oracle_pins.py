@@ -460,7 +460,8 @@ def test_round_bf16_is_round_to_nearest_even():
 @pytest.mark.parametrize("kind", KINDS)
 def test_keys_backward_with_bf16_operands_matches_dense(kind):
     """operand_bf16=True equals the dense definition with P and dS rounded to
-    bf16 (explicit mask, union softmax, dense products)."""
+    bf16 and D taken from the bf16-rounded O (explicit mask, union softmax,
+    dense products)."""
     st = wl.random_structure(23, n_seqs=2, max_len=20, max_depth=4, hq=4, hkv=2, head_dim=8,
                              mask_kind=kind, branch_prob=0.6)
     t = _f64_tensors(st, 5)
@@ -480,7 +481,7 @@ def test_keys_backward_with_bf16_operands_matches_dense(kind):
         s = np.where(mask, s, -np.inf)
         lse = np.log(np.exp(s - s.max(1, keepdims=True)).sum(1)) + s.max(1)
         p = np.where(mask, np.exp(s - lse[:, None]), 0.0)
-        o = p @ v[:, g]
+        o = oracle.round_bf16(p @ v[:, g])          # the forward's bf16 output
         ds = p * (do[:, h] @ v[:, g].T - (do[:, h] * o).sum(1)[:, None])
         dv[:, g] += oracle.round_bf16(p).T @ do[:, h]
         dk[:, g] += st.scale * oracle.round_bf16(ds).T @ q[:, h]
