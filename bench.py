@@ -162,18 +162,22 @@ class ClockSampler:
                 "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
 
 
-# The sources that decide what the profiled launches do: the tcgen05 kernels
-# and their headers, the backward preprocess, the plan (work order) and the
-# dispatch.  Host staging (step_host.cu) and the static-scratch entry do not
-# change those launches.
-PROFILED_SOURCES = ("api.cu", "attn_sm100.cu", "attn_sm100_bwd.cu", "attn_sm100_common.cuh",
-                    "internal.cuh", "merge.cu", "plan.cu", "sm100.cuh")
+# The sources that decide what a profiled launch does, per profile kind: the
+# attention kernels with their headers, the plan (tile ranges and work order)
+# and the launch configuration.  Host staging, the static-scratch entry, the
+# ring entry points and the streaming kernels do not change those launches.
+PROFILED_SOURCES = {
+    "fwd_attention": ("attn_sm100.cu", "attn_sm100_common.cuh", "internal.cuh", "plan.cu",
+                      "sm100.cuh"),
+    "bwd_attention": ("attn_sm100_bwd.cu", "attn_sm100_common.cuh", "internal.cuh", "plan.cu",
+                      "sm100.cuh"),
+}
 
 
-def kernel_source_sha():
+def kernel_source_sha(kernel: str = "bwd_attention"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "speculative_draft_branch_b200", "csrc")
-    for f in PROFILED_SOURCES:
+    for f in PROFILED_SOURCES[kernel]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -188,7 +192,7 @@ def profiled_traffic(kernel: str, workload: str):
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     s = re.search(r"source_sha:\s*([0-9a-f]+)", text)
-    if not m or not s or s.group(1) != kernel_source_sha():
+    if not m or not s or s.group(1) != kernel_source_sha(kernel):
         return None
     return float(m.group(1))
 

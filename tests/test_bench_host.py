@@ -128,11 +128,12 @@ def test_clock_sampler_without_nvidia_smi(monkeypatch):
 
 def test_profiled_traffic_only_for_the_profiled_sources(monkeypatch):
     """The traffic figure of a profile summary is used only while its source
-    hash matches the current kernel sources."""
+    hash matches the current kernel sources; every profile kind hashes its own
+    list of sources, and every listed file exists."""
     import tempfile
     sys.path.insert(0, ROOT)
     import bench
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "00c0ffee00c0ffee")
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda kernel="bwd_attention": "00c0ffee00c0ffee")
     os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
     with tempfile.TemporaryDirectory(dir=os.path.join(ROOT, "_build")) as tmp:
         os.mkdir(os.path.join(tmp, "profiles"))
@@ -144,3 +145,6 @@ def test_profiled_traffic_only_for_the_profiled_sources(monkeypatch):
         assert bench.profiled_traffic("bwd_attention", "w") == 2.5e9
         assert bench.profiled_traffic("fwd_attention", "w") is None     # stale profile
         assert bench.profiled_traffic("bwd_attention", "other") is None  # no profile
+    monkeypatch.undo()
+    for kind in bench.PROFILED_SOURCES:
+        assert len(bench.kernel_source_sha(kind)) == 16
