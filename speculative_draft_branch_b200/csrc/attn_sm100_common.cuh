@@ -25,50 +25,60 @@ struct Seg {
   int key0, n, kind, full_b, full_e;
 };
 
+// Up to three key segments of a query tile, walked in order.  Kept as three
+// named members (never an array indexed at run time), so the walk stays in
+// registers instead of local memory.
 struct TileSegs {
-  Seg s[3];
+  Seg s0, s1, s2;
   int total;
   __device__ __forceinline__ void locate(int it, int &key0, int &kind, bool &full) const {
-    int si = 0, sub = it;
-    if (sub >= s[0].n) {
-      sub -= s[0].n;
-      si = 1;
-      if (sub >= s[1].n) {
-        sub -= s[1].n;
-        si = 2;
+    int sub = it;
+    Seg g = s0;
+    if (sub >= s0.n) {
+      sub -= s0.n;
+      g = s1;
+      if (sub >= s1.n) {
+        sub -= s1.n;
+        g = s2;
       }
     }
-    const Seg g = si == 0 ? s[0] : (si == 1 ? s[1] : s[2]);
     key0 = g.key0 + sub * 128;
     kind = g.kind;
     full = kind == 0 && key0 >= g.full_b && key0 + 128 <= g.full_e;
+  }
+  __device__ __forceinline__ void push(const Seg &g, int &n) {
+    if (n == 0) s0 = g;
+    else if (n == 1) s1 = g;
+    else s2 = g;
+    ++n;
   }
 };
 
 __device__ __forceinline__ TileSegs make_segs(const AttnParams &a, int t, bool is_main) {
   TileSegs ts;
+  const Seg none = {0, 0, 2, 0, 0};
+  ts.s0 = none; ts.s1 = none; ts.s2 = none;
   int n = 0;
   const int32_t *qt = a.plan.qtile + (int64_t)t * 6;
   const int zz = a.zz_step;
   if (zz < 0 || (a.ring && zz < a.zz_C)) {
     const int k0 = qt[0] * 128, k1 = min(qt[3] * 128, a.n_keys_m);
-    if (k1 > k0) ts.s[n++] = {k0, (k1 - k0 + 127) / 128, 0, qt[1] * 128, qt[2] * 128};
+    if (k1 > k0) ts.push({k0, (k1 - k0 + 127) / 128, 0, qt[1] * 128, qt[2] * 128}, n);
   } else if (zz < a.zz_C) {
     const int32_t *z = a.plan.zz_tiles + ((int64_t)zz * a.n_qt + t) * 4;
+#pragma unroll
     for (int w = 0; w < 2; ++w) {
       const int k0 = z[2 * w] * 128, k1 = min(z[2 * w + 1] * 128, a.n_keys_m);
-      if (k1 > k0) ts.s[n++] = {k0, (k1 - k0 + 127) / 128, w, 0, 0};
+      if (k1 > k0) ts.push({k0, (k1 - k0 + 127) / 128, w, 0, 0}, n);
     }
   }
   if (!is_main && (zz < 0 || zz == a.zz_C)) {
     const int b0 = qt[4], b1 = qt[5];
-    if (b1 > b0) ts.s[n++] = {b0, (b1 - b0 + 127) / 128, 2, 0, 0};
+    if (b1 > b0) ts.push({b0, (b1 - b0 + 127) / 128, 2, 0, 0}, n);
   }
-  for (int i = n; i < 3; ++i) ts.s[i] = {0, 0, 2, 0, 0};
-  ts.total = ts.s[0].n + ts.s[1].n + ts.s[2].n;
+  ts.total = ts.s0.n + ts.s1.n + ts.s2.n;
   return ts;
 }
-
 
 // ---- key-stationary backward walk -------------------------------------------
 constexpr int kQc = 128;  // query rows per chunk: N of the S^T / dP^T products
