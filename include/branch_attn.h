@@ -340,6 +340,68 @@ BA_API ba_status branch_attn_ring_finish(const ba_problem *local, int32_t C, con
                                          void *o_m, void *o_b, float *lse_m, float *lse_b,
                                          ba_stream_t stream);
 
+/* ---- TapChannel: target features across pipeline stages ---------------------
+ * The method-detail section's pipeline transport (and the technical
+ * contribution's mailboxes, sequence stamps and pre-allocated slots): stages
+ * that compute target features write them straight into slots the draft's
+ * stage allocated beforehand, outside the pipeline's schedule, and the
+ * consumer reads a slot once its sequence stamp shows the message it expects.
+ * Within a node the mailbox is shared through CUDA IPC (the producer's copy
+ * engine writes over NVLink when the consumer is another GPU).
+ *
+ * The consumer owns one device region, the mailbox (ba_tap_mailbox_size
+ * bytes: stamps and acks [n_producers][n_slots] int64, then the slots).
+ * Message `seq` of producer p travels through slot seq mod n_slots:
+ *   - ba_tap_send (producer) waits on the host until that slot's previous
+ *     message (seq - n_slots) has been released, copies the payload into the
+ *     slot on `stream` and then writes the stamp, in stream order;
+ *   - ba_tap_wait (consumer) polls the stamp on the host until it equals seq
+ *     and returns the slot's device address;
+ *   - ba_tap_release (consumer) marks the slot free on `stream`, after the
+ *     work that reads it.
+ * No kernel ever waits for another process; every wait is a host poll bounded
+ * by timeout_ns (BA_ERR_DEVICE_TIMEOUT when it runs out).  Producers and the
+ * consumer may run on different GPUs of a node or on the same one. */
+typedef struct ba_tap ba_tap;
+
+/* Bytes of a mailbox: n_producers in [1, 256], n_slots in [1, 1024],
+ * slot_bytes a positive multiple of 16.  Host-only. */
+BA_API ba_status ba_tap_mailbox_size(int32_t n_producers, int32_t n_slots, int64_t slot_bytes,
+                                     size_t *bytes);
+
+/* Consumer side: turns caller-owned device memory (`mailbox`, 256-byte
+ * aligned, at least ba_tap_mailbox_size bytes, on the current device) into a
+ * channel, clears its stamps and acks (synchronising the device) and writes
+ * into handle_out (at least 128 bytes) the blob producers attach with; the
+ * caller hands it to them (any byte transport).  *out must be released with
+ * ba_tap_close; the mailbox memory stays the caller's. */
+BA_API ba_status ba_tap_create(void *mailbox, size_t mailbox_bytes, int32_t n_producers,
+                               int32_t n_slots, int64_t slot_bytes, void *handle_out,
+                               size_t handle_bytes, ba_tap **out);
+
+/* Producer side: maps the consumer's mailbox (CUDA IPC, in another process)
+ * as producer `producer`, on the current device. */
+BA_API ba_status ba_tap_attach(const void *handle, size_t handle_bytes, int32_t producer,
+                               ba_tap **out);
+
+/* Producer: message seq (>= 0, consecutive per producer) of `bytes` (at most
+ * the slot size) from device memory `src`; returns once the copy and the
+ * stamp are enqueued on `stream` (src must stay unchanged until then). */
+BA_API ba_status ba_tap_send(ba_tap *t, int64_t seq, const void *src, int64_t bytes,
+                             int64_t timeout_ns, ba_stream_t stream);
+
+/* Consumer: waits for message seq of `producer`; *slot receives its device
+ * address (valid until ba_tap_release). */
+BA_API ba_status ba_tap_wait(ba_tap *t, int32_t producer, int64_t seq, int64_t timeout_ns,
+                             void **slot);
+
+/* Consumer: frees the slot of message seq of `producer` once `stream` reaches
+ * this point. */
+BA_API ba_status ba_tap_release(ba_tap *t, int32_t producer, int64_t seq, ba_stream_t stream);
+
+/* Either side: unmaps (producer) and frees the channel object. */
+BA_API ba_status ba_tap_close(ba_tap *t);
+
 /* Device self-check of the exponentials available to the softmax (no
  * counterpart in the paper): the hardware ex2 unit the kernels use, and a
  * range-reduced cubic on the FMA pipe (max relative error 7.5e-5) kept as an

@@ -34,7 +34,8 @@ EXPORTS = ("ba_workspace_size", "ba_plan_layout_query", "ba_plan", "ba_plan_stat
            "ba_version", "branch_attn_bwd_static_scratch", "ba_exp2_check",
            "ba_step_host_workspace_size", "branch_attn_step_host", "ba_wait_check",
            "ba_zigzag_shard", "ba_ring_workspace_size", "ba_ring_plan", "branch_attn_ring_step",
-           "branch_attn_ring_finish")
+           "branch_attn_ring_finish", "ba_tap_mailbox_size", "ba_tap_create", "ba_tap_attach",
+           "ba_tap_send", "ba_tap_wait", "ba_tap_release", "ba_tap_close")
 
 
 class BAProblem(ctypes.Structure):
@@ -90,6 +91,13 @@ def _load() -> ctypes.CDLL:
         "ba_ring_plan": [P, I32, I32, I32, VP, VP, VP, S, VP],
         "branch_attn_ring_step": [P, I32, I32, VP, VP, S, I32, VP, VP, VP, VP, VP],
         "branch_attn_ring_finish": [P, I32, VP, VP, S] + [VP] * 8 + [VP],
+        "ba_tap_mailbox_size": [I32, I32, I64, ctypes.POINTER(S)],
+        "ba_tap_create": [VP, S, I32, I32, I64, VP, S, ctypes.POINTER(VP)],
+        "ba_tap_attach": [VP, S, I32, ctypes.POINTER(VP)],
+        "ba_tap_send": [VP, I64, VP, I64, I64, VP],
+        "ba_tap_wait": [VP, I32, I64, I64, ctypes.POINTER(VP)],
+        "ba_tap_release": [VP, I32, I64, VP],
+        "ba_tap_close": [VP],
         "ba_launch_count": [],
         "ba_last_error": [],
         "ba_version": [],
@@ -456,6 +464,69 @@ def branch_attn_ring_finish(local: Problem, C: int, plan_ws, acc_ws, q_m, q_b, k
         ctypes.byref(local.c), C, _ptr(plan_ws), _ptr(acc_ws),
         acc_ws.numel() * acc_ws.element_size(), _ptr(q_m), _ptr(q_b), _ptr(k_b), _ptr(v_b),
         _ptr(o_m), _ptr(o_b), _ptr(lse_m), _ptr(lse_b), _stream(stream)))
+
+
+# ---- TapChannel ---------------------------------------------------------------
+TAP_HANDLE_BYTES = 128
+
+
+def ba_tap_mailbox_size(n_producers: int, n_slots: int, slot_bytes: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib.ba_tap_mailbox_size(n_producers, n_slots, slot_bytes, ctypes.byref(n)))
+    return n.value
+
+
+class TapConsumer:
+    """The draft stage's end of a TapChannel: owns the mailbox (device memory
+    allocated here with torch) and hands out `handle`, the bytes producers
+    attach with."""
+
+    def __init__(self, n_producers: int, n_slots: int, slot_bytes: int, device="cuda"):
+        import torch
+        self.n_producers, self.n_slots, self.slot_bytes = n_producers, n_slots, slot_bytes
+        nbytes = ba_tap_mailbox_size(n_producers, n_slots, slot_bytes)
+        self.mailbox = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        blob = ctypes.create_string_buffer(TAP_HANDLE_BYTES)
+        t = ctypes.c_void_p()
+        _check(lib.ba_tap_create(self.mailbox.data_ptr(), nbytes, n_producers, n_slots,
+                                 slot_bytes, blob, TAP_HANDLE_BYTES, ctypes.byref(t)))
+        self._t, self.handle = t, blob.raw
+
+    def wait(self, producer: int, seq: int, timeout_s: float = 10.0):
+        """Message `seq` of `producer` as a uint8 view of its slot."""
+        p = ctypes.c_void_p()
+        _check(lib.ba_tap_wait(self._t, producer, seq, int(timeout_s * 1e9), ctypes.byref(p)))
+        off = p.value - self.mailbox.data_ptr()
+        return self.mailbox[off:off + self.slot_bytes]
+
+    def release(self, producer: int, seq: int, stream=None) -> None:
+        _check(lib.ba_tap_release(self._t, producer, seq, _stream(stream)))
+
+    def close(self) -> None:
+        if self._t:
+            _check(lib.ba_tap_close(self._t))
+            self._t = None
+
+
+class TapProducer:
+    """A producer stage's end: maps the consumer's mailbox from its handle."""
+
+    def __init__(self, handle: bytes, producer: int):
+        t = ctypes.c_void_p()
+        buf = ctypes.create_string_buffer(bytes(handle), len(handle))
+        _check(lib.ba_tap_attach(buf, len(handle), producer, ctypes.byref(t)))
+        self._t, self.producer = t, producer
+
+    def send(self, seq: int, src, timeout_s: float = 10.0, stream=None) -> None:
+        """Message `seq` from the CUDA tensor `src` (contiguous, current device)."""
+        _expect_ws(src, "src")
+        _check(lib.ba_tap_send(self._t, seq, src.data_ptr(), src.numel() * src.element_size(),
+                               int(timeout_s * 1e9), _stream(stream)))
+
+    def close(self) -> None:
+        if self._t:
+            _check(lib.ba_tap_close(self._t))
+            self._t = None
 
 
 def ba_set_kernel_family(family: int) -> None:
