@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(384, 1)
 // dK / dV kernel
 // ============================================================================
 constexpr int kQStages = 2;   // Q ring (freed once dK of the chunk is done)
-constexpr int kDoStages = 2;  // dO + records ring (freed once dV of the chunk is done)
+constexpr int kDoStages = 2;  // dO + records ring (freed once dK of the chunk, after its dS work, is issued)
 
 template <int D>
 struct DkvSmem {
@@ -354,7 +354,7 @@ struct DkvSmem {
   uint64_t bar_kv;
   uint64_t bar_q_full[kQStages], bar_q_empty[kQStages];
   uint64_t bar_do_full[kDoStages], bar_do_empty[kDoStages];
-  uint64_t bar_s_full, bar_x_free, bar_dp_full, bar_pds_full;
+  uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready;
   uint64_t bar_acc_done;
   uint64_t bar_drain;
   uint32_t tmem_base;
@@ -363,12 +363,15 @@ struct DkvSmem {
 
 // TMEM columns: dK [0, D), dV [D, 2D), X = S^T at 2D, Y = dP^T at 2D + 128
 // (128 columns each).  Four threads per key row, one per query quarter
-// [32 qq, 32 qq + 32) (16 warps; warp w reaches TMEM lanes 32 (w % 4) ..):
-// each reads its S^T quarter from X (freeing X for the next chunk's S^T as
-// soon as every thread has it in registers), then reads dP^T from Y and
-// writes P^T and dS^T (bf16 pairs, 16 columns each) over the 32 columns it
-// read.  K-step k (queries 16k..16k+15) of the dV product reads P^T at
-// Y + 32 (k / 2) + 8 (k % 2), that of the dK product dS^T 16 columns further.
+// [32 qq, 32 qq + 32) (16 warps; warp w reaches TMEM lanes 32 (w % 4) ..).
+// Each thread writes only over the 32 columns of X and Y it has read itself:
+// P^T (bf16 pairs, 16 columns) over its S^T quarter in X as soon as the
+// exponentials are done, dS^T over its dP^T quarter in Y once dP^T is there.
+// K-step k (queries 16k..16k+15) of the dV product reads P^T at
+// X + 32 (k / 2) + 8 (k % 2), that of the dK product dS^T at the same offset
+// in Y.  So dV(c) waits only for the exponentials of chunk c, not for dP^T(c)
+// and the dS work: issue order per chunk dV(c), S^T(c+1), dK(c), dP^T(c+1),
+// and the dS work of chunk c runs under dV(c) and S^T(c+1).
 // 576 threads: warp 0 producer, warp 1 MMA issuer, warps 2-17 P^T / dS^T.
 constexpr int kDkvThreads = 576;
 constexpr int kDkvElem = kDkvThreads - 64;   // P^T / dS^T threads
@@ -394,8 +397,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   volatile int *abort_flag = &sm.abort_flag;
 
   const uint32_t b_kv = smem_u32(&sm.bar_kv), b_acc = smem_u32(&sm.bar_acc_done);
-  const uint32_t b_s = smem_u32(&sm.bar_s_full), b_xf = smem_u32(&sm.bar_x_free);
-  const uint32_t b_dp = smem_u32(&sm.bar_dp_full), b_pds = smem_u32(&sm.bar_pds_full);
+  const uint32_t b_s = smem_u32(&sm.bar_s_full), b_pr = smem_u32(&sm.bar_p_ready);
+  const uint32_t b_dp = smem_u32(&sm.bar_dp_full), b_dsr = smem_u32(&sm.bar_ds_ready);
   if (threadIdx.x == 0) {
     mbar_init(b_kv, 1);
     for (int s = 0; s < kQStages; ++s) {
@@ -407,9 +410,9 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       mbar_init(smem_u32(&sm.bar_do_empty[s]), 1);
     }
     mbar_init(b_s, 1);
-    mbar_init(b_xf, kDkvElem);
+    mbar_init(b_pr, kDkvElem);
     mbar_init(b_dp, 1);
-    mbar_init(b_pds, kDkvElem);
+    mbar_init(b_dsr, kDkvElem);
     mbar_init(b_acc, 1);
     mbar_init(smem_u32(&sm.bar_drain), 1);
     sm.abort_flag = 0;
@@ -479,71 +482,84 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     if (total > 0) mbar_wait_drain(b_kv, 0, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    // Issue order per chunk c: S^T(c+1), dK(c), dV(c), dP^T(c+1).  S^T(c+1)
-    // overwrites X once the P^T threads hold S^T(c); dP^T(c+1) overwrites Y
-    // after dK(c) / dV(c) have read P^T and dS^T from it: tcgen05 MMAs issued
-    // by one thread run in order.
+    // Issue order per chunk c: dV(c), S^T(c+1), dK(c), dP^T(c+1).  S^T(c+1)
+    // overwrites X after dV(c) has read P^T(c) from it, dP^T(c+1) overwrites Y
+    // after dK(c) has read dS^T(c): tcgen05 MMAs issued by one thread run in
+    // order.  Waits are grouped (a wait in this thread holds it until its
+    // queued MMAs are nearly done): before dV(c) for P^T(c) and Q(c+1),
+    // before dK(c) for dS^T(c) and dO(c+1).
     constexpr uint32_t idesc_s = idesc_bf16(128, kQc, false, false);
     constexpr uint32_t idesc_g = idesc_bf16(128, D, false, true);
     bool ok = total == 0 || mbar_wait(b_kv, 0, abort_flag, status_word, 3);
     const uint64_t kd0 = sdesc(smem_u32(sm.k), 16, 1024), vd0 = sdesc(smem_u32(sm.v), 16, 1024);
-    auto issue_s = [&](int c) -> bool {
-      const int st = c % kQStages;
-      if (!mbar_wait(smem_u32(&sm.bar_q_full[st]), (c / kQStages) & 1, abort_flag, status_word,
-                     5))
-        return false;
-      if (c > 0 && !mbar_wait(b_xf, (c - 1) & 1, abort_flag, status_word, 6)) return false;
-      tc_fence_after();
-      const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16, 1024);
+    auto wait_q = [&](int c) -> bool {
+      return mbar_wait(smem_u32(&sm.bar_q_full[c % kQStages]), (c / kQStages) & 1, abort_flag,
+                       status_word, 5);
+    };
+    auto wait_do = [&](int c) -> bool {
+      return mbar_wait(smem_u32(&sm.bar_do_full[c % kDoStages]), (c / kDoStages) & 1, abort_flag,
+                       status_word, 5);
+    };
+    auto issue_s = [&](int c) {
+      const uint64_t qd = sdesc(smem_u32(sm.q[c % kQStages]), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
         mma_bf16(t_x, desc_at(kd0, off), desc_at(qd, off), idesc_s, k > 0 ? 1u : 0u);
       }
       mma_commit(b_s);
-      return true;
     };
-    auto issue_dp = [&](int c) -> bool {
-      const int ds = c % kDoStages;
-      if (!mbar_wait(smem_u32(&sm.bar_do_full[ds]), (c / kDoStages) & 1, abort_flag, status_word,
-                     5))
-        return false;
-      tc_fence_after();
-      const uint64_t dd = sdesc(smem_u32(sm.dout[ds]), 16, 1024);
+    auto issue_dp = [&](int c) {
+      const uint64_t dd = sdesc(smem_u32(sm.dout[c % kDoStages]), 16, 1024);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
         mma_bf16(t_y, desc_at(vd0, off), desc_at(dd, off), idesc_s, k > 0 ? 1u : 0u);
       }
       mma_commit(b_dp);
-      return true;
     };
-    auto issue_grads = [&](int c) -> bool {
-      if (!mbar_wait(b_pds, c & 1, abort_flag, status_word, 4)) return false;
-      tc_fence_after();
+    if (ok && total > 0) {
+      ok = wait_q(0) && wait_do(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      }
+    }
+    for (int c = 0; ok && c < total; ++c) {
       const int st = c % kQStages, ds = c % kDoStages;
+      const uint32_t acc = c > 0 ? 1u : 0u;
       // B operands MN-major: K = 16 queries per step (16 rows of 128 B), the
       // two 64-column halves of D one 16 KB box apart
-      const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16384, 1024);
+      if (!mbar_wait(b_pr, c & 1, abort_flag, status_word, 4) || (c + 1 < total && !wait_q(c + 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
       const uint64_t dd = sdesc(smem_u32(sm.dout[ds]), 16384, 1024);
-      // dK += dS^T Q, then dV += P^T dO (K = 128 queries)
+      // dV += P^T dO (P^T from X)
 #pragma unroll
       for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16_ts(t_dk, t_y + (k >> 1) * 32 + 16 + (k & 1) * 8, desc_at(qd, k * 2048), idesc_g,
-                    (c > 0 || k > 0) ? 1u : 0u);
+        mma_bf16_ts(t_dv, t_x + (k >> 1) * 32 + (k & 1) * 8, desc_at(dd, k * 2048), idesc_g,
+                    (acc | (uint32_t)k) ? 1u : 0u);
+      if (c + 1 < total) issue_s(c + 1);
+      if (!mbar_wait(b_dsr, c & 1, abort_flag, status_word, 6) ||
+          (c + 1 < total && !wait_do(c + 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint64_t qd = sdesc(smem_u32(sm.q[st]), 16384, 1024);
+      // dK += dS^T Q (dS^T from Y)
+#pragma unroll
+      for (int k = 0; k < kQc / 16; ++k)
+        mma_bf16_ts(t_dk, t_y + (k >> 1) * 32 + (k & 1) * 8, desc_at(qd, k * 2048), idesc_g,
+                    (acc | (uint32_t)k) ? 1u : 0u);
       mma_commit(smem_u32(&sm.bar_q_empty[st]));
-#pragma unroll
-      for (int k = 0; k < kQc / 16; ++k)
-        mma_bf16_ts(t_dv, t_y + (k >> 1) * 32 + (k & 1) * 8, desc_at(dd, k * 2048), idesc_g,
-                    (c > 0 || k > 0) ? 1u : 0u);
+      // the dO stage also holds chunk c's records, read by the dS work that
+      // ds_ready(c) waited for: free it only now (dV(c) ran before in order)
       mma_commit(smem_u32(&sm.bar_do_empty[ds]));
-      return true;
-    };
-    if (ok && total > 0) ok = issue_s(0) && issue_dp(0);
-    for (int c = 0; ok && c < total; ++c) {
-      if (c + 1 < total && !issue_s(c + 1)) ok = false;
-      else if (!issue_grads(c)) ok = false;
-      else if (c + 1 < total && !issue_dp(c + 1)) ok = false;
+      if (c + 1 < total) issue_dp(c + 1);
     }
     if (ok && total > 0) mma_commit(b_acc);
     mma_commit(smem_u32(&sm.bar_drain));
@@ -573,11 +589,10 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
         break;
       }
       tc_fence_after();
+      const uint32_t colx = t_x + lane_addr + qq * 32, coly = t_y + lane_addr + qq * 32;
       float p[32];
-      tmem_ld32(t_x + lane_addr + qq * 32, reinterpret_cast<uint32_t *>(p));
+      tmem_ld32(colx, reinterpret_cast<uint32_t *>(p));
       tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive(b_xf);
       // the records come with dO
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_do_full[ds]), (c / kDoStages) & 1,
                                              abort_flag, status_word, 8))) {
@@ -595,26 +610,30 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       }
 #pragma unroll
       for (int q = 0; q < 32; ++q) p[q] = ex2(fmaf(p[q], sl2, -rec[q].x));
+      // P^T over this thread's own S^T columns: dV(c) may start now
+      uint32_t pk[16];
+#pragma unroll
+      for (int q = 0; q < 32; q += 2) pk[q / 2] = pack_bf16(p[q], p[q + 1]);
+      tmem_st16(colx, pk);
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(b_pr);
       if (!__all_sync(0xffffffffu, mbar_wait(b_dp, c & 1, abort_flag, status_word, 9))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t col = t_y + lane_addr + qq * 32;
       float dp[32];
-      tmem_ld32(col, reinterpret_cast<uint32_t *>(dp));
+      tmem_ld32(coly, reinterpret_cast<uint32_t *>(dp));
       tc_wait_ld();
-      uint32_t pk[16], dk2[16];
+      uint32_t dk2[16];
 #pragma unroll
-      for (int q = 0; q < 32; q += 2) {
-        pk[q / 2] = pack_bf16(p[q], p[q + 1]);
+      for (int q = 0; q < 32; q += 2)
         dk2[q / 2] = pack_bf16(p[q] * (dp[q] - rec[q].y), p[q + 1] * (dp[q + 1] - rec[q + 1].y));
-      }
-      tmem_st16(col, pk);
-      tmem_st16(col + 16, dk2);
+      tmem_st16(coly, dk2);
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(b_pds);
+      mbar_arrive(b_dsr);
     }
     if (ok && total > 0 &&
         !__all_sync(0xffffffffu, mbar_wait(b_acc, 0, abort_flag, status_word, 10)))
