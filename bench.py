@@ -828,7 +828,7 @@ def run_tap_bench(args):
     max over producers of their device time (CUDA events on each producer's
     stream).  Host staging: device -> pinned host -> device of the same
     bytes, CUDA events on one stream.  Contention: branch_attn_fwd on the TTT
-    20K batch alone and while 64 MB writes land in the receiver's memory from
+    20K batch alone and while 256 MB writes land in the receiver's memory from
     a side stream at the full device copy rate."""
     import multiprocessing as mp
 
@@ -837,7 +837,7 @@ def run_tap_bench(args):
     import speculative_draft_branch_b200 as ba
     import workloads as wl
     P = args.tap_bench
-    n_msg, nbytes, n_slots = 16, 64 << 20, 4
+    n_msg, nbytes, n_slots = 8, 256 << 20, 4
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     ctx = mp.get_context("spawn")
@@ -909,7 +909,7 @@ def run_tap_bench(args):
     feed = torch.randint(0, 255, (nbytes,), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
     with torch.cuda.stream(side):
-        for _ in range(3000):
+        for _ in range(2500):
             inbox.copy_(feed, non_blocking=True)
     under = fwd_ms(20)
     side_busy = not side.query()        # the writes outlasted the timed forwards
@@ -925,7 +925,7 @@ def run_tap_bench(args):
                                 "writes_covered_the_timing": side_busy},
         "note": "producers and consumer share one GPU: the channel's copies stay inside one "
                 "GPU's HBM (no NVLink); host staging crosses the host link twice; the "
-                "receiver's slowdown is measured under 64 MB device-to-device writes into its "
+                "receiver's slowdown is measured under 256 MB device-to-device writes into its "
                 "memory from a side stream at full copy rate (an upper bound on incoming "
                 "feature traffic)"}))
     return 0
