@@ -794,9 +794,9 @@ def run_shard_timing(args):
 
 
 # ---------------------------------------------------------------- TapChannel
-def _tap_producer(handle, producer, n_msg, nbytes, q):
-    """One producer stage: sends n_msg messages of nbytes through the channel;
-    reports its device time from before the first send to after the last."""
+def _tap_producer(handle, producer, n_msg, nbytes, q, go):
+    """One producer stage: once every producer is ready and the consumer has
+    started its clock, sends n_msg messages of nbytes through the channel."""
     import torch
 
     import speculative_draft_branch_b200 as ba
@@ -804,15 +804,15 @@ def _tap_producer(handle, producer, n_msg, nbytes, q):
     try:
         tx = ba.TapProducer(handle, producer)
         src = torch.randint(0, 255, (nbytes,), dtype=torch.uint8, device="cuda")
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        e0.record()
+        q.put((producer, "ready"))
+        if not go.wait(timeout=300):
+            raise TimeoutError("no start signal")
         for seq in range(n_msg):
             tx.send(seq, src, timeout_s=120)
-        e1.record()
         torch.cuda.synchronize()
         tx.close()
-        q.put((producer, e0.elapsed_time(e1)))
+        q.put((producer, "done"))
     except Exception as e:
         q.put((producer, repr(e)))
 
@@ -825,9 +825,11 @@ def run_tap_bench(args):
     Producers run as processes on the same GPU as the consumer (one GPU per
     call here), so the channel's copies are device-to-device within one GPU's
     HBM rather than over NVLink.  Fan-in rate: bytes of all messages over the
-    max over producers of their device time (CUDA events on each producer's
-    stream).  Host staging: device -> pinned host -> device of the same
-    bytes, CUDA events on one stream.  Contention: branch_attn_fwd on the TTT
+    consumer's wall time from the common start signal to the stamp of the
+    last message (the consumer releases each slot as it arrives, so producers
+    wait for free slots as they would in a pipeline).  Host staging: device ->
+    pinned host -> device of the same bytes, CUDA events on one stream (a
+    lower bound on that path: no host synchronisation counted).  Contention: branch_attn_fwd on the TTT
     20K batch alone and while 256 MB writes land in the receiver's memory from
     a side stream at the full device copy rate."""
     import multiprocessing as mp
@@ -844,23 +846,30 @@ def run_tap_bench(args):
 
     def fan_in():
         rx = ba.TapConsumer(P, n_slots, nbytes, dev)
-        q = ctx.Queue()
-        procs = [ctx.Process(target=_tap_producer, args=(rx.handle, p, n_msg, nbytes, q))
+        q, go = ctx.Queue(), ctx.Event()
+        procs = [ctx.Process(target=_tap_producer, args=(rx.handle, p, n_msg, nbytes, q, go))
                  for p in range(P)]
         for p in procs:
             p.start()
+        ready = [q.get(timeout=300) for _ in procs]
+        if any(r[1] != "ready" for r in ready):
+            go.set()
+            raise RuntimeError(f"producer failed: {ready}")
+        t0 = time.perf_counter()
+        go.set()
         for seq in range(n_msg):
             for p in range(P):
                 rx.wait(p, seq, timeout_s=300)
                 rx.release(p, seq)
+        ms = (time.perf_counter() - t0) * 1e3
         res = [q.get(timeout=300) for _ in procs]
         for p in procs:
             p.join(timeout=120)
         rx.close()
-        bad = [r for r in res if not isinstance(r[1], float)]
+        bad = [r for r in res if r[1] != "done"]
         if bad:
             raise RuntimeError(f"producer failed: {bad}")
-        return max(r[1] for r in res)
+        return ms
 
     ms_ipc = fan_in()
     total = P * n_msg * nbytes
@@ -888,37 +897,48 @@ def run_tap_bench(args):
     runner.plan()
     out = runner.alloc_outputs()
 
-    def fwd_ms(n):
-        ms = []
+    side = torch.cuda.Stream(device=dev)
+    inbox = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    feed = torch.randint(0, 255, (nbytes,), dtype=torch.uint8, device=dev)
+    side_end = torch.cuda.Event()
+
+    def fwd_ms(n, feed_copies=0):
+        """Median forward time over n launches.  With feed_copies, each launch
+        is preceded by that many 256 MB writes into the receiver's memory on
+        a side stream (enough to outlast the launch); the wait is on the
+        forward's own end event, so the side stream keeps running."""
+        ms, covered = [], True
         for _ in range(n):
+            if feed_copies:
+                with torch.cuda.stream(side):
+                    for _ in range(feed_copies):
+                        inbox.copy_(feed, non_blocking=True)
+                    side_end.record(side)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             runner.forward(t, out)
             b.record()
-            torch.cuda.synchronize()
+            b.synchronize()
+            if feed_copies:
+                covered = covered and not side_end.query()
             ms.append(a.elapsed_time(b))
-        return statistics.median(ms)
+        torch.cuda.synchronize()
+        return statistics.median(ms), covered
 
     fwd_ms(3)
-    alone = fwd_ms(20)
+    alone, _ = fwd_ms(20)
     # incoming writes into the receiver's memory at the full device copy rate,
     # from a side stream of this process (other processes would be time-sliced
     # against this one on a shared GPU, which is not what a receiver sees)
-    side = torch.cuda.Stream(device=dev)
-    inbox = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    feed = torch.randint(0, 255, (nbytes,), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
-    with torch.cuda.stream(side):
-        for _ in range(2500):
-            inbox.copy_(feed, non_blocking=True)
-    under = fwd_ms(20)
-    side_busy = not side.query()        # the writes outlasted the timed forwards
-    torch.cuda.synchronize()
+    under, side_busy = fwd_ms(20, feed_copies=64)
     print(json.dumps({
         "study": "tap_channel", "producers": P, "messages_per_producer": n_msg,
         "message_bytes": nbytes, "slots": n_slots,
-        "fan_in": {"ms": ms_ipc, "GB_per_s": total / (ms_ipc * 1e-3) / 1e9},
-        "host_staging": {"ms": ms_host, "GB_per_s": total / (ms_host * 1e-3) / 1e9},
+        "fan_in": {"ms": ms_ipc, "GB_per_s": total / (ms_ipc * 1e-3) / 1e9,
+                   "timing": "consumer wall clock, start signal to last stamp"},
+        "host_staging": {"ms": ms_host, "GB_per_s": total / (ms_host * 1e-3) / 1e9,
+                         "timing": "CUDA events, copies only"},
         "speedup_over_host_staging": ms_host / ms_ipc,
         "receiver_forward_ms": {"alone": alone, "under_incoming_writes": under,
                                 "slowdown": under / alone - 1.0,

@@ -374,7 +374,7 @@ ba_status branch_attn_bwd(const ba_problem *p, const void *plan_ws, void *bwd_ws
   a.dk_b = (__nv_bfloat16 *)dk_b; a.dv_b = (__nv_bfloat16 *)dv_b;
   char *ws = reinterpret_cast<char *>(bwd_ws);
   a.d_all = reinterpret_cast<const float *>(ws);
-  a.rec = reinterpret_cast<float4 *>(ws + bwd_d_bytes(*p));
+  a.rec = reinterpret_cast<float *>(ws + bwd_d_bytes(*p));
   a.dq_acc = reinterpret_cast<float *>(ws + bwd_d_bytes(*p) + bwd_rec_bytes(*p));
   a.n_main_pad = (int32_t)align_up((size_t)p->n_main, 128);
   a.rows_pad = (int32_t)rows_padded(*p);

@@ -12,7 +12,7 @@
 // Two kernels, neither with atomics:
 //   dq_sm100_kernel    query-stationary (one CTA per 128-row query tile and q
 //                      head, the forward's work order): per key tile S and dP
-//                      into TMEM, dS by 256 threads (two per row) written back
+//                      into TMEM, dS by 512 threads (four per row) written back
 //                      to TMEM as bf16, dQ += dS K (A operand from TMEM)
 //                      accumulated in TMEM; K and V come through separate
 //                      rings so V is refilled as soon as dP is done.  S / dP
@@ -66,9 +66,15 @@ struct DqMaps {
 };
 
 // TMEM columns: S [0, 128), dP [128, 256), dQ [256, 256 + D), dS (bf16 pairs)
-// double-buffered at 384 and 448.
+// double-buffered at 384 and 448.  608 threads: warp 0 producer, warp 1 S / dP
+// issuer, warp 2 TMEM owner and dQ issuer, warps 3-18 dS, four threads per
+// query row (warp w reaches TMEM lanes 32 (w % 4) .., key quarter
+// (w - 3) / 4 of the tile).
+constexpr int kDqThreads = 608;
+constexpr int kDqElem = kDqThreads - 96;
+
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     dq_sm100_kernel(const AttnParams a, const __grid_constant__ DqMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -104,9 +110,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(smem_u32(&sm.bar_v_empty[s]), 1);
     }
     mbar_init(b_sdp_full, 1);
-    mbar_init(b_sdp_empty, 256);
-    mbar_init(smem_u32(&sm.bar_ds_full[0]), 256);
-    mbar_init(smem_u32(&sm.bar_ds_full[1]), 256);
+    mbar_init(b_sdp_empty, kDqElem);
+    mbar_init(smem_u32(&sm.bar_ds_full[0]), kDqElem);
+    mbar_init(smem_u32(&sm.bar_ds_full[1]), kDqElem);
     mbar_init(smem_u32(&sm.bar_dq_done[0]), 1);
     mbar_init(smem_u32(&sm.bar_dq_done[1]), 1);
     mbar_init(b_final, 1);
@@ -172,7 +178,7 @@ __global__ void __launch_bounds__(384, 1)
     if (total > 0) mbar_wait_drain(b_qdo, 0, status_word, 2);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ S / dP issuer
-    // Two issuing threads: this one issues S and dP of each key tile, warp 3
+    // Two issuing threads: this one issues S and dP of each key tile, warp 2
     // the dQ products.  An mbarrier wait holds the thread that executes it
     // until the MMAs it has queued are done, so one issuer waiting for dS
     // would keep the next tile's S / dP out of the tensor pipe (and waiting
@@ -209,7 +215,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     mma_commit(smem_u32(&sm.bar_drain[0]));
     mbar_wait_drain(smem_u32(&sm.bar_drain[0]), 0, status_word, 2);
-  } else if (warp == 3 && lane == 0) {
+  } else if (warp == 2 && lane == 0) {
     // ------------------------------------------------------------ dQ issuer
     // dQ(i) += dS(i) K(i).  K(i) is released here: S(i) read it before the
     // dS threads could finish tile i.
@@ -232,11 +238,10 @@ __global__ void __launch_bounds__(384, 1)
     if (ok && total > 0) mma_commit(b_final);
     mma_commit(smem_u32(&sm.bar_drain[1]));
     mbar_wait_drain(smem_u32(&sm.bar_drain[1]), 0, status_word, 2);
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ dS (2 threads / row)
-    const int ew = threadIdx.x - 128;
-    const int half = ew >> 7;
-    const int row = ew & 127;
+  } else if (warp >= 3) {
+    // ------------------------------------------------------------ dS (4 threads / row)
+    const int qq = (warp - 3) >> 2;  // key quarter [32 qq, 32 qq + 32) of each tile
+    const int row = (warp & 3) * 32 + lane;
     const bool valid = row < nrows;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     int lo0 = 0, hi0 = -1, lo2 = 0, hi2 = -1;
@@ -258,20 +263,18 @@ __global__ void __launch_bounds__(384, 1)
       bool full;
       segs.locate(j, key0, kind, full);
       const int clo = kind == 2 ? lo2 : lo0, chi = kind == 2 ? hi2 : hi0;
-      float s[64], dp[64];
-      tmem_ld32(t_s + lane_addr + half * 64, reinterpret_cast<uint32_t *>(s));
-      tmem_ld32(t_s + lane_addr + half * 64 + 32, reinterpret_cast<uint32_t *>(s) + 32);
-      tmem_ld32(t_dp + lane_addr + half * 64, reinterpret_cast<uint32_t *>(dp));
-      tmem_ld32(t_dp + lane_addr + half * 64 + 32, reinterpret_cast<uint32_t *>(dp) + 32);
+      float s[32], dp[32];
+      tmem_ld32(t_s + lane_addr + qq * 32, reinterpret_cast<uint32_t *>(s));
+      tmem_ld32(t_dp + lane_addr + qq * 32, reinterpret_cast<uint32_t *>(dp));
       tc_wait_ld();
       tc_fence_before();
       mbar_arrive(b_sdp_empty);
-      const int kbase = key0 + half * 64;
+      const int kbase = key0 + qq * 32;
       // masked scores -> -inf only on partial tiles, then P = 2^(s sl2 - l2)
       // branch-free; dS packed to bf16 pairs in place (entry c/2 after c, c+1)
       if (!(full && valid)) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < 32; ++c) {
           const int key = kbase + c;
           if (key < clo || key > chi) s[c] = kNegInf;
         }
@@ -279,7 +282,7 @@ __global__ void __launch_bounds__(384, 1)
       const float sl2 = a.scale_log2;
       uint32_t *pk = reinterpret_cast<uint32_t *>(dp);
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         float d2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -296,7 +299,7 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       tc_fence_after();
-      tmem_st32(t_ds(j & 1) + lane_addr + half * 32, pk);
+      tmem_st16(t_ds(j & 1) + lane_addr + qq * 16, pk);
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.bar_ds_full[j & 1]));
@@ -305,22 +308,23 @@ __global__ void __launch_bounds__(384, 1)
         !__all_sync(0xffffffffu, mbar_wait(b_final, 0, abort_flag, status_word, 9)))
       ok = false;
     tc_fence_after();
+    // each of the four threads of a row stores a quarter of its dQ
+    constexpr int kCols = D / 4;
     bf16 *dst = (is_main ? a.dq_out_m : a.dq_out_b) + ((int64_t)(row0 + row) * a.hq + h) * D +
-                half * (D / 2);
+                qq * kCols;
+    uint32_t o[kCols];
+    if (ok && total > 0) {
+      if constexpr (kCols == 32) tmem_ld32(t_dq + lane_addr + qq * kCols, o);
+      else tmem_ld16(t_dq + lane_addr + qq * kCols, o);
+      tc_wait_ld();
+    } else {
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      uint32_t o[32];
-      if (ok && total > 0) {
-        tmem_ld32(t_dq + lane_addr + half * (D / 2) + c * 32, o);
-        tc_wait_ld();
-      } else {
+      for (int e = 0; e < kCols; ++e) o[e] = 0u;
+    }
+    if (valid) {
+      uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = 0u;
-      }
-      if (!valid) continue;
-      uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
+      for (int e = 0; e < kCols / 8; ++e)
         d4[e] = make_uint4(
             pack_bf16(__uint_as_float(o[8 * e]) * a.scale, __uint_as_float(o[8 * e + 1]) * a.scale),
             pack_bf16(__uint_as_float(o[8 * e + 2]) * a.scale,
@@ -335,7 +339,10 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, 512);
+  if (warp == 2) {
+    __syncwarp();  // lane 0 comes back from the dQ issuer's loop
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 // ============================================================================
@@ -350,7 +357,8 @@ struct DkvSmem {
   bf16 v[128 * D];
   bf16 q[kQStages][kQc * D];      // D/64 boxes of [128 rows][64], 16 KB each
   bf16 dout[kDoStages][kQc * D];
-  float4 rec[kDoStages][kQc];     // {LSE log2, D, key lo, key hi} per query
+  alignas(16) float rec[kDoStages][4 * kQc];  // LSE log2[128], D[128], key lo[128], key hi[128]
+  int chunk_full[kDoStages];      // every query of the chunk sees every key of the tile
   uint64_t bar_kv;
   uint64_t bar_q_full[kQStages], bar_q_empty[kQStages];
   uint64_t bar_do_full[kDoStages], bar_do_empty[kDoStages];
@@ -428,7 +436,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const uint32_t t_dk = tmem, t_dv = tmem + D, t_x = tmem + 2 * D, t_y = tmem + 2 * D + 128;
   // records of this CTA's key kind: main-key intervals or branch-local ones
-  const float4 *rec_base = a.rec + (main_kv ? 0 : (int64_t)a.hq * a.rows_pad);
+  const int64_t rec_kind = main_kv ? 0 : a.hq;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -464,6 +472,15 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
           !mbar_wait(smem_u32(&sm.bar_do_empty[ds]), ((c / kDoStages) - 1) & 1, abort_flag,
                      status_word, 1))
         break;
+      // a chunk whose every query sees every key of this tile needs no mask;
+      // the flag travels with the stage (published by the arrive below)
+      bool full = false;
+      if (main_kv) {
+        const int32_t *qt =
+            a.plan.qtile + (int64_t)(is_main_q ? tile : a.n_qt_main + tile) * 6;
+        full = nrows == kQc && kt >= qt[1] && kt < qt[2];
+      }
+      sm.chunk_full[ds] = full ? 1 : 0;
       const uint32_t dbar = smem_u32(&sm.bar_do_full[ds]);
       mbar_expect_tx(dbar, kQc * D * 2 + kQc * 16);
       const CUtensorMap *dm = is_main_q ? &tm.do_m : &tm.do_b;
@@ -471,7 +488,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       for (int x = 0; x < D / 64; ++x)
         tma_load_3d(smem_u32(sm.dout[ds]) + x * 16384, dm, dbar, x * 64, h, row0);
       const int64_t prow = (is_main_q ? 0 : a.n_main_pad) + row0;
-      bulk_load(smem_u32(sm.rec[ds]), rec_base + (int64_t)h * a.rows_pad + prow, kQc * 16, dbar);
+      bulk_load(smem_u32(sm.rec[ds]), a.rec + rec_block(rec_kind + h, a.rows_pad, prow), kQc * 16,
+                dbar);
       ++do_issued;
     }
     // no copy may still be writing shared memory when the CTA exits
@@ -574,16 +592,6 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     bool ok = true;
     for (int c = 0; c < total; ++c) {
       const int ds = c % kDoStages;
-      // a chunk whose every query sees every key of this tile needs no mask
-      bool full = false;
-      if (main_kv) {
-        int h, tile, nrows;
-        bool is_main_q;
-        cw.at(c, a, h, is_main_q, tile, nrows);
-        const int32_t *qt =
-            a.plan.qtile + (int64_t)(is_main_q ? tile : a.n_qt_main + tile) * 6;
-        full = nrows == kQc && kt >= qt[1] && kt < qt[2];
-      }
       if (!__all_sync(0xffffffffu, mbar_wait(b_s, c & 1, abort_flag, status_word, 7))) {
         ok = false;
         break;
@@ -599,17 +607,29 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
         ok = false;
         break;
       }
-      const float4 *rec = sm.rec[ds] + qq * 32;
-      if (!full) {
+      // this quarter's 32 queries of each record field, four per 16-byte load
+      const float4 *r_lse = reinterpret_cast<const float4 *>(sm.rec[ds] + kRecLse + qq * 32);
+      const float4 *r_d = reinterpret_cast<const float4 *>(sm.rec[ds] + kRecD + qq * 32);
+      if (!sm.chunk_full[ds]) {
+        const int4 *r_lo = reinterpret_cast<const int4 *>(sm.rec[ds] + kRecLo + qq * 32);
+        const int4 *r_hi = reinterpret_cast<const int4 *>(sm.rec[ds] + kRecHi + qq * 32);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int2 iv =
-              *reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(&rec[q]) + 8);
-          if (key < iv.x || key > iv.y) p[q] = kNegInf;
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const int4 lo = r_lo[q4], hi = r_hi[q4];
+          if (key < lo.x || key > hi.x) p[4 * q4] = kNegInf;
+          if (key < lo.y || key > hi.y) p[4 * q4 + 1] = kNegInf;
+          if (key < lo.z || key > hi.z) p[4 * q4 + 2] = kNegInf;
+          if (key < lo.w || key > hi.w) p[4 * q4 + 3] = kNegInf;
         }
       }
 #pragma unroll
-      for (int q = 0; q < 32; ++q) p[q] = ex2(fmaf(p[q], sl2, -rec[q].x));
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 l = r_lse[q4];
+        p[4 * q4] = ex2(fmaf(p[4 * q4], sl2, -l.x));
+        p[4 * q4 + 1] = ex2(fmaf(p[4 * q4 + 1], sl2, -l.y));
+        p[4 * q4 + 2] = ex2(fmaf(p[4 * q4 + 2], sl2, -l.z));
+        p[4 * q4 + 3] = ex2(fmaf(p[4 * q4 + 3], sl2, -l.w));
+      }
       // P^T over this thread's own S^T columns: dV(c) may start now
       uint32_t pk[16];
 #pragma unroll
@@ -628,8 +648,12 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       tc_wait_ld();
       uint32_t dk2[16];
 #pragma unroll
-      for (int q = 0; q < 32; q += 2)
-        dk2[q / 2] = pack_bf16(p[q] * (dp[q] - rec[q].y), p[q + 1] * (dp[q + 1] - rec[q + 1].y));
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 dd = r_d[q4];
+        dk2[2 * q4] = pack_bf16(p[4 * q4] * (dp[4 * q4] - dd.x), p[4 * q4 + 1] * (dp[4 * q4 + 1] - dd.y));
+        dk2[2 * q4 + 1] =
+            pack_bf16(p[4 * q4 + 2] * (dp[4 * q4 + 2] - dd.z), p[4 * q4 + 3] * (dp[4 * q4 + 3] - dd.w));
+      }
       tmem_st16(coly, dk2);
       tc_wait_st();
       tc_fence_before();
@@ -723,13 +747,13 @@ ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s) {
     if ((st = launch_kernel(dkdv_sm100_kernel<64>, sizeof(DkvSmem<64>) + 1024, grid_kv, kDkvThreads, a,
                             kvm, s, "dkdv_sm100_kernel<64>")) != BA_OK)
       return st;
-    return launch_kernel(dq_sm100_kernel<64>, sizeof(DqSmem<64>) + 1024, grid_dq, 384, a, dqm, s,
+    return launch_kernel(dq_sm100_kernel<64>, sizeof(DqSmem<64>) + 1024, grid_dq, kDqThreads, a, dqm, s,
                          "dq_sm100_kernel<64>");
   }
   if ((st = launch_kernel(dkdv_sm100_kernel<128>, sizeof(DkvSmem<128>) + 1024, grid_kv, kDkvThreads, a,
                           kvm, s, "dkdv_sm100_kernel<128>")) != BA_OK)
     return st;
-  return launch_kernel(dq_sm100_kernel<128>, sizeof(DqSmem<128>) + 1024, grid_dq, 384, a, dqm, s,
+  return launch_kernel(dq_sm100_kernel<128>, sizeof(DqSmem<128>) + 1024, grid_dq, kDqThreads, a, dqm, s,
                        "dq_sm100_kernel<128>");
 }
 

@@ -46,7 +46,8 @@ struct FusedSmem {
   bf16 q[2][kQc * D];
   bf16 dout[2][kQc * D];
   bf16 ds[128 * kQc];              // dS^T: two boxes [128 keys][64 queries]
-  float4 rec[kQc];
+  alignas(16) float rec[4 * kQc];  // LSE log2[128], D[128], key lo[128], key hi[128]
+  int rec_full;                     // every query of the chunk sees every key of the tile
   uint64_t bar_kv;
   uint64_t bar_q_full[2], bar_q_empty[2];
   uint64_t bar_do_full[2], bar_do_empty[2];
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const uint32_t t_dk = tmem, t_dv = tmem + D, t_sp = tmem + 2 * D, t_qb = tmem + 2 * D + 128;
   // records of this CTA's key kind: main-key intervals or branch-local ones
-  const float4 *rec_base = a.rec + (main_kv ? 0 : (int64_t)a.hq * a.rows_pad);
+  const int64_t rec_kind = main_kv ? 0 : a.hq;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -165,9 +166,19 @@ __global__ void __launch_bounds__(kFThreads, 1)
       ++do_issued;
       // the single record buffer is free once chunk c-1's elementwise work is done
       if (c >= 1 && !mbar_wait(b_pds, (c - 1) & 1, abort_flag, status_word, 1)) break;
+      // a chunk whose every query sees every key of this tile needs no mask;
+      // the flag is published by the arrive below, with the records
+      bool full = false;
+      if (main_kv) {
+        const int32_t *qt =
+            a.plan.qtile + (int64_t)(is_main_q ? tile : a.n_qt_main + tile) * 6;
+        full = nrows == kQc && kt >= qt[1] && kt < qt[2];
+      }
+      sm.rec_full = full ? 1 : 0;
       mbar_expect_tx(b_rec, kQc * 16);
       const int64_t prow = (is_main_q ? 0 : a.n_main_pad) + row0;
-      bulk_load(smem_u32(sm.rec), rec_base + (int64_t)h * a.rows_pad + prow, kQc * 16, b_rec);
+      bulk_load(smem_u32(sm.rec), a.rec + rec_block(rec_kind + h, a.rows_pad, prow), kQc * 16,
+                b_rec);
       ++rec_issued;
     }
     // no copy may still be writing shared memory when the CTA exits
@@ -309,16 +320,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
       return true;
     };
     for (int c = 0; c < total; ++c) {
-      // a chunk whose every query sees every key of this tile needs no mask
-      bool full = false;
-      if (main_kv) {
-        int h, tile, nrows;
-        bool is_main_q;
-        cw.at(c, a, h, is_main_q, tile, nrows);
-        const int32_t *qt =
-            a.plan.qtile + (int64_t)(is_main_q ? tile : a.n_qt_main + tile) * 6;
-        full = nrows == kQc && kt >= qt[1] && kt < qt[2];
-      }
       // ---- exp phase: S^T(c) -> P
       if (!__all_sync(0xffffffffu, mbar_wait(b_s, c & 1, abort_flag, status_word, 7))) {
         ok = false;
@@ -334,17 +335,29 @@ __global__ void __launch_bounds__(kFThreads, 1)
         ok = false;
         break;
       }
-      const float4 *rec = sm.rec + qq * 32;
-      if (!full) {
+      // this quarter's 32 queries of each record field, four per 16-byte load
+      const float4 *r_lse = reinterpret_cast<const float4 *>(sm.rec + kRecLse + qq * 32);
+      const float4 *r_d = reinterpret_cast<const float4 *>(sm.rec + kRecD + qq * 32);
+      if (!sm.rec_full) {
+        const int4 *r_lo = reinterpret_cast<const int4 *>(sm.rec + kRecLo + qq * 32);
+        const int4 *r_hi = reinterpret_cast<const int4 *>(sm.rec + kRecHi + qq * 32);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int2 iv =
-              *reinterpret_cast<const int2 *>(reinterpret_cast<const char *>(&rec[q]) + 8);
-          if (key < iv.x || key > iv.y) p[q] = kNegInf;
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const int4 lo = r_lo[q4], hi = r_hi[q4];
+          if (key < lo.x || key > hi.x) p[4 * q4] = kNegInf;
+          if (key < lo.y || key > hi.y) p[4 * q4 + 1] = kNegInf;
+          if (key < lo.z || key > hi.z) p[4 * q4 + 2] = kNegInf;
+          if (key < lo.w || key > hi.w) p[4 * q4 + 3] = kNegInf;
         }
       }
 #pragma unroll
-      for (int q = 0; q < 32; ++q) p[q] = ex2(fmaf(p[q], sl2, -rec[q].x));
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 l = r_lse[q4];
+        p[4 * q4] = ex2(fmaf(p[4 * q4], sl2, -l.x));
+        p[4 * q4 + 1] = ex2(fmaf(p[4 * q4 + 1], sl2, -l.y));
+        p[4 * q4 + 2] = ex2(fmaf(p[4 * q4 + 2], sl2, -l.z));
+        p[4 * q4 + 3] = ex2(fmaf(p[4 * q4 + 3], sl2, -l.w));
+      }
       uint32_t pk[16];
 #pragma unroll
       for (int q = 0; q < 32; q += 2) pk[q / 2] = pack_bf16(p[q], p[q + 1]);
@@ -367,8 +380,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
       tmem_st16(col, pk);
       uint32_t dk2[16];
 #pragma unroll
-      for (int q = 0; q < 32; q += 2)
-        dk2[q / 2] = pack_bf16(p[q] * (dp[q] - rec[q].y), p[q + 1] * (dp[q + 1] - rec[q + 1].y));
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 dd = r_d[q4];
+        dk2[2 * q4] = pack_bf16(p[4 * q4] * (dp[4 * q4] - dd.x), p[4 * q4 + 1] * (dp[4 * q4 + 1] - dd.y));
+        dk2[2 * q4 + 1] =
+            pack_bf16(p[4 * q4 + 2] * (dp[4 * q4 + 2] - dd.z), p[4 * q4 + 3] * (dp[4 * q4 + 3] - dd.w));
+      }
       // row `row` of dS^T, queries [32 qq, 32 qq + 32): 16-byte chunks
       // (qq & 1) * 4 + e of the row, placed by the 128-byte swizzle
 #pragma unroll

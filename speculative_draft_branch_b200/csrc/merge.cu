@@ -99,11 +99,12 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, int heads,
 // ---- backward preprocess ---------------------------------------------------
 // D[h, row] = sum_d dO[row, h, d] * O[row, h, d] (fp32 accumulate), rows =
 // main rows then branch rows, and the per-query records the backward reads
-// {l log2 e, D, key lo, key hi} (main-key interval and branch-local interval).
+// {l log2 e, D, key lo, key hi} (main-key interval and branch-local interval),
+// laid out as four arrays of 128 per 128-row block.
 // A warp takes 32 consecutive rows of one head, one lane per row: each lane
 // streams its row's 2 d bf16 of O and dO (16-byte loads, all issued before
-// the products), and the warp's writes of D and of the records are 128- and
-// 512-byte contiguous runs.  When the backward accumulates dQ in fp32 the
+// the products), and the warp's writes of D and of each record field are
+// 128-byte contiguous runs.  When the backward accumulates dQ in fp32 the
 // accumulator of the same row-head is zeroed in the same pass.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(AttnParams a) {
@@ -149,9 +150,10 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(AttnParams a) {
                      1.4426950408889634f;
     const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[row];
     const int64_t pr = (is_main ? 0 : a.n_main_pad) + r;
-    a.rec[(int64_t)h * a.rows_pad + pr] = make_float4(l2, s, __int_as_float(iv.x), __int_as_float(iv.y));
-    a.rec[((int64_t)a.hq + h) * a.rows_pad + pr] =
-        make_float4(l2, s, __int_as_float(iv.z), __int_as_float(iv.w));
+    float *r0 = a.rec + rec_block(h, a.rows_pad, pr) + (pr & 127);
+    float *r1 = a.rec + rec_block((int64_t)a.hq + h, a.rows_pad, pr) + (pr & 127);
+    r0[kRecLse] = l2; r0[kRecD] = s; r0[kRecLo] = __int_as_float(iv.x); r0[kRecHi] = __int_as_float(iv.y);
+    r1[kRecLse] = l2; r1[kRecD] = s; r1[kRecLo] = __int_as_float(iv.z); r1[kRecHi] = __int_as_float(iv.w);
   }
   // padding rows of the records: empty key intervals
   const int pad_m = a.n_main_pad - a.n_main;
@@ -163,7 +165,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(AttnParams a) {
     const int64_t kh = i / per;
     const int j = (int)(i % per);
     const int64_t pr = j < pad_m ? a.n_main + j : a.n_main_pad + a.n_bt + (j - pad_m);
-    a.rec[kh * a.rows_pad + pr] = make_float4(0.f, 0.f, __int_as_float(1), __int_as_float(0));
+    float *rp = a.rec + rec_block(kh, a.rows_pad, pr) + (pr & 127);
+    rp[kRecLse] = 0.f; rp[kRecD] = 0.f; rp[kRecLo] = __int_as_float(1); rp[kRecHi] = __int_as_float(0);
   }
 }
 
