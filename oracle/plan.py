@@ -18,6 +18,8 @@ this library's contract, written in the plain per-tile form:
       tiles: [0, 0));
   * per query row: the closed interval of visible main keys and of visible
     branch-local key rows (empty = [0, -1]), read off the mask definition;
+  * per key row: the main query rows and the branch query rows that see it,
+    each a half-open row range (empty = [0, 0));
   * per main key tile k: the main and the branch query tiles t with
     kv_begin(t) <= k < kv_end(t), as index ranges (empty = [0, 0));
   * per branch key tile k' (rows [k' BN, (k'+1) BN)): the branch query tiles
@@ -66,6 +68,43 @@ def row_intervals(st) -> np.ndarray:
             out[n:, 3] = dv.cu_branch[b + 1] - 1
         else:
             out[n:, 3] = np.arange(nb)
+    return out
+
+
+def _interval_of_rows(lo: np.ndarray, hi: np.ndarray, keys: np.ndarray) -> np.ndarray:
+    """For each key k: the query rows r with lo[r] <= k <= hi[r], as
+    [begin, end) (empty = (0, 0)); returns [len(keys), 2].
+
+    lo and hi are non-decreasing over the rows (asserted by the caller), so
+    {r : hi[r] >= k} is a suffix and {r : lo[r] <= k} a prefix, and their
+    intersection is the interval between the two boundaries.
+    """
+    b = np.searchsorted(hi, keys, side="left")
+    e = np.searchsorted(lo, keys, side="right")
+    empty = b >= e
+    return np.stack([np.where(empty, 0, b), np.where(empty, 0, e)], axis=1).astype(np.int64)
+
+
+def key_intervals(st) -> np.ndarray:
+    """[(N + Nb), 4] int64 per key row: the main query rows that see it as
+    [begin, end), then the branch query rows (indexed from 0 over the branch
+    rows) as [begin, end); empty = (0, 0).  Main keys first, then branch keys,
+    which only branch rows see (through their branch-local interval).
+
+    Follows from the per-row intervals (row_intervals): main rows and branch
+    rows each have non-decreasing lower and upper bounds (rows in packed order,
+    anchors non-decreasing), so the rows seeing one key are contiguous.
+    """
+    iv = row_intervals(st)
+    n, nb = st.n_main, st.n_branch_tokens
+    m, b = iv[:n], iv[n:]
+    for part in (m[:, 0], m[:, 1], b[:, 0], b[:, 1], b[:, 2], b[:, 3]):
+        assert np.all(np.diff(part) >= 0), "row bounds must be non-decreasing"
+    out = np.zeros((n + nb, 4), dtype=np.int64)
+    main_keys, branch_keys = np.arange(n), np.arange(nb)
+    out[:n, :2] = _interval_of_rows(m[:, 0], m[:, 1], main_keys)
+    out[:n, 2:] = _interval_of_rows(b[:, 0], b[:, 1], main_keys)
+    out[n:, 2:] = _interval_of_rows(b[:, 2], b[:, 3], branch_keys)
     return out
 
 
@@ -121,6 +160,7 @@ def plan(st, BM: int = PLAN_BM, BN: int = PLAN_BN) -> dict:
         "cu_branch": dv.cu_branch.copy(),
         "branch_seq": dv.branch_seq.copy(),
         "row_iv": row_intervals(st),
+        "key_iv": key_intervals(st),
         "qtile": qt,
         "kv_main": kv_main,
         "kv_branch": kv_branch,

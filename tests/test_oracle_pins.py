@@ -323,6 +323,16 @@ def test_plan_matches_bruteforce(kind, seed, tile):
             assert lk.size == lk.max() - lk.min() + 1
         else:
             assert tuple(iv[r, 2:]) == (0, -1)
+    # per-key intervals: the mask column's main rows and branch rows, each
+    # exactly the listed half-open range
+    ki = p["key_iv"]
+    for k in range(n + nb):
+        col = mask[:, k]
+        for part, (lo_r, hi_r) in ((slice(0, 2), (0, n)), (slice(2, 4), (n, n + nb))):
+            rows = np.nonzero(col[lo_r:hi_r])[0]
+            want = (int(rows.min()), int(rows.max()) + 1) if rows.size else (0, 0)
+            assert tuple(ki[k, part]) == want, (k, part)
+            assert rows.size == want[1] - want[0]
     n_mt = -(-n // BM)
     qt = p["qtile"]
     tiles = [(0, t * BM, min((t + 1) * BM, n)) for t in range(n_mt)]
