@@ -318,10 +318,9 @@ def hbm_steps(ba, runner, t, out, grads, stream, dev, hbm_gbs, max_rows=1 << 18)
 
     D preprocess: launched inside branch_attn_bwd ahead of the attention
     kernels; the library records a pair of CUDA events right around it.  Per
-    (row, head) it reads O and dO (2 d bf16) and the LSE and writes D and two
-    16-byte records; per row it reads the 16-byte key interval; with the fused
-    backward (family 1) it also zeroes the fp32 dQ accumulator, 4 d bytes per
-    row and head."""
+    (row, head) it reads O and dO (2 d bf16) and the LSE and writes D and the
+    8-byte record {LSE log2 e, D}; with the fused backward (family 1) it also
+    zeroes the fp32 dQ accumulator, 4 d bytes per row and head."""
     import torch
     c = runner.problem.c
     rows, heads, d = c.n_main + c.n_branch_tokens, c.hq, c.head_dim
@@ -371,7 +370,7 @@ def hbm_steps(ba, runner, t, out, grads, stream, dev, hbm_gbs, max_rows=1 << 18)
     finally:
         ba.ba_set_kernel_events(2, None, None)
     zero_acc = 4 * d if ba.ba_get_kernel_family() == 1 else 0
-    res["bwd_preprocess"] = roof(rows * heads * (2 * d * 2 + 4 + 4 + 32 + zero_acc) + rows * 16,
+    res["bwd_preprocess"] = roof(rows * heads * (2 * d * 2 + 4 + 4 + 8 + zero_acc),
                                  statistics.median(times),
                                  note="CUDA events on the launching stream around the "
                                       "preprocess kernel alone (median of 3 launches)")

@@ -134,14 +134,19 @@ typedef struct {
  *   bwd_order   [n_kv_main + n_kv_branch]  key tiles by decreasing cost
  *   fwd_cost, bwd_cost           the costs used for the two orders
  *   zz_tiles    [zigzag_C * n_qtiles * 4]  (zigzag_C > 1 only) per ring step
- *               and query tile, two key-tile ranges [b0, e0), [b1, e1)  */
+ *               and query tile, two key-tile ranges [b0, e0), [b1, e1)
+ *   key_iv      [(n_main + n_branch_tokens) * 4]  per key row (main keys
+ *               first): the main query rows that see it [x, y) and the branch
+ *               query rows that see it [z, w) (branch rows counted from 0);
+ *               empty = (0, 0).  Contiguous because row bounds are
+ *               non-decreasing; used by the backward's key-stationary walk. */
 #define BA_TILE_M 128
 #define BA_TILE_N 128
 typedef struct {
   size_t total_bytes;
   size_t off_status, off_cu_branch, off_branch_seq, off_row_iv, off_qtile;
   size_t off_kv_main, off_kv_branch, off_fwd_order, off_bwd_order;
-  size_t off_fwd_cost, off_bwd_cost, off_zz_tiles;
+  size_t off_fwd_cost, off_bwd_cost, off_zz_tiles, off_key_iv;
   int32_t n_qtiles_main, n_qtiles_branch, n_kv_main, n_kv_branch;
 } ba_plan_layout;
 
@@ -151,9 +156,9 @@ typedef struct {
  * fwd_bytes:  scratch of branch_attn_fwd (0 when zigzag_C == 1; otherwise
  *   fp32 accumulators of O and LSE for every query row and head).
  * bwd_bytes:  scratch of branch_attn_bwd: D = rowsum(dO * O) fp32
- *   [Hq, rows], per-query records {LSE log2 e, D, first key, last key}
- *   (float4, twice per row and head, rows padded to 128 per token kind) and
- *   the fp32 dQ accumulator [rows, Hq, d] of the fused backward. */
+ *   [Hq, rows], per-query records {LSE log2 e, D} (8 bytes per row and head,
+ *   rows padded to 128 per token kind) and the fp32 dQ accumulator
+ *   [rows, Hq, d] of the fused backward. */
 BA_API ba_status ba_workspace_size(const ba_problem *p, size_t *plan_bytes,
                             size_t *fwd_bytes, size_t *bwd_bytes);
 

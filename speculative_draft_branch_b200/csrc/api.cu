@@ -130,6 +130,7 @@ void plan_layout(const ba_problem &p, ba_plan_layout *L) {
   L->off_fwd_cost = take(4 * (size_t)n_qt);
   L->off_bwd_cost = take(4 * (size_t)n_kv);
   L->off_zz_tiles = take(p.zigzag_C > 1 ? 16 * (size_t)p.zigzag_C * n_qt : 0);
+  L->off_key_iv = take(16 * (size_t)rows);
   L->total_bytes = off;
 }
 
@@ -148,6 +149,7 @@ PlanView plan_view(const ba_plan_layout &L, const void *ws) {
   v.fwd_cost = reinterpret_cast<int32_t *>(b + L.off_fwd_cost);
   v.bwd_cost = reinterpret_cast<int32_t *>(b + L.off_bwd_cost);
   v.zz_tiles = reinterpret_cast<int32_t *>(b + L.off_zz_tiles);
+  v.key_iv = reinterpret_cast<int32_t *>(b + L.off_key_iv);
   return v;
 }
 
@@ -168,7 +170,7 @@ size_t rows_padded(const ba_problem &p) {
 size_t bwd_d_bytes(const ba_problem &p) {
   return align_up(4 * ((size_t)p.n_main + p.n_branch_tokens) * p.hq, 256);
 }
-size_t bwd_rec_bytes(const ba_problem &p) { return align_up(2 * 16 * rows_padded(p) * p.hq, 256); }
+size_t bwd_rec_bytes(const ba_problem &p) { return align_up(8 * rows_padded(p) * p.hq, 256); }
 size_t bwd_ws_bytes(const ba_problem &p) {
   const size_t rows = (size_t)p.n_main + p.n_branch_tokens;
   return bwd_d_bytes(p) + bwd_rec_bytes(p) + align_up(4 * rows * p.hq * p.head_dim, 256);

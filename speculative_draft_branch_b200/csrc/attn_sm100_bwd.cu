@@ -25,10 +25,11 @@
 //                      TMEM (N = 128: the tensor cores' full rate), P^T and
 //                      dS^T written over dP^T as bf16, dV += P^T dO and
 //                      dK += dS^T Q (A operands from TMEM) accumulated in TMEM
-//                      for the whole walk.  Q and dO come through separate
-//                      two-deep rings, each freed by the product that reads it
-//                      last; per-query records {LSE, D, key interval} arrive by
-//                      bulk copy with dO.
+//                      for the whole walk.  Q (three deep) and dO (two deep)
+//                      come through separate rings, each freed by the product
+//                      that reads it last; per-query records {LSE, D} arrive by
+//                      bulk copy with dO; each key thread masks with the plan's
+//                      range of query rows that see its key.
 #include "attn_sm100_common.cuh"
 
 namespace ba {
@@ -348,7 +349,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 // ============================================================================
 // dK / dV kernel
 // ============================================================================
-constexpr int kQStages = 2;   // Q ring (freed once dK of the chunk is done)
+// Q(c + 1) is read by S^T(c + 1), issued right after dV(c); Q(c - 1), whose
+// stage it would take in a two-deep ring, is freed only by dK(c - 1): three deep.
+constexpr int kQStages = 3;
 constexpr int kDoStages = 2;  // dO + records ring (freed once dK of the chunk, after its dS work, is issued)
 
 template <int D>
@@ -357,8 +360,8 @@ struct DkvSmem {
   bf16 v[128 * D];
   bf16 q[kQStages][kQc * D];      // D/64 boxes of [128 rows][64], 16 KB each
   bf16 dout[kDoStages][kQc * D];
-  alignas(16) float rec[kDoStages][4 * kQc];  // LSE log2[128], D[128], key lo[128], key hi[128]
-  int chunk_full[kDoStages];      // every query of the chunk sees every key of the tile
+  alignas(16) float rec[kDoStages][2 * kQc];  // LSE log2 [128], D [128]
+  int4 chunk[kDoStages];          // {no mask needed, branch query tile, first query row}
   uint64_t bar_kv;
   uint64_t bar_q_full[kQStages], bar_q_empty[kQStages];
   uint64_t bar_do_full[kDoStages], bar_do_empty[kDoStages];
@@ -368,6 +371,7 @@ struct DkvSmem {
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(DkvSmem<128>) <= 232448, "dK/dV kernel exceeds 227 KB of shared memory");
 
 // TMEM columns: dK [0, D), dV [D, 2D), X = S^T at 2D, Y = dP^T at 2D + 128
 // (128 columns each).  Four threads per key row, one per query quarter
@@ -388,9 +392,15 @@ template <int D>
 __global__ void __launch_bounds__(kDkvThreads, 1)
     dkdv_sm100_kernel(const AttnParams a, const __grid_constant__ DkvMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  DkvSmem<D> &sm = *reinterpret_cast<DkvSmem<D> *>(smem_raw + (((raw + 1023) & ~1023u) - raw));
+  DkvSmem<D> &sm = *reinterpret_cast<DkvSmem<D> *>(smem_raw);
   if (a.plan.status[0] != 0) return;
+  int *status_word = a.plan.status + 1;
+  // the 128-byte swizzled tiles need 1024-byte aligned shared memory; the
+  // layout has no room for padding, so refuse (status bit 14) instead
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(status_word, 1 << 14);
+    return;
+  }
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int item = a.plan.bwd_order[blockIdx.x / a.hkv];
@@ -401,7 +411,6 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   const int n_keys = main_kv ? a.n_main : a.n_bt;
   const ChunkWalk cw = make_walk(a, main_kv, kt, g);
   const int total = cw.grp * (cw.n_t0 + cw.n_t1);
-  int *status_word = a.plan.status + 1;
   volatile int *abort_flag = &sm.abort_flag;
 
   const uint32_t b_kv = smem_u32(&sm.bar_kv), b_acc = smem_u32(&sm.bar_acc_done);
@@ -435,8 +444,6 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const uint32_t t_dk = tmem, t_dv = tmem + D, t_x = tmem + 2 * D, t_y = tmem + 2 * D + 128;
-  // records of this CTA's key kind: main-key intervals or branch-local ones
-  const int64_t rec_kind = main_kv ? 0 : a.hq;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -473,23 +480,23 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
                      status_word, 1))
         break;
       // a chunk whose every query sees every key of this tile needs no mask;
-      // the flag travels with the stage (published by the arrive below)
+      // the chunk's description travels with the stage (published by the
+      // arrive below)
       bool full = false;
       if (main_kv) {
         const int32_t *qt =
             a.plan.qtile + (int64_t)(is_main_q ? tile : a.n_qt_main + tile) * 6;
         full = nrows == kQc && kt >= qt[1] && kt < qt[2];
       }
-      sm.chunk_full[ds] = full ? 1 : 0;
+      sm.chunk[ds] = make_int4(full ? 1 : 0, is_main_q ? 0 : 1, row0, 0);
       const uint32_t dbar = smem_u32(&sm.bar_do_full[ds]);
-      mbar_expect_tx(dbar, kQc * D * 2 + kQc * 16);
+      mbar_expect_tx(dbar, kQc * D * 2 + kQc * 8);
       const CUtensorMap *dm = is_main_q ? &tm.do_m : &tm.do_b;
 #pragma unroll
       for (int x = 0; x < D / 64; ++x)
         tma_load_3d(smem_u32(sm.dout[ds]) + x * 16384, dm, dbar, x * 64, h, row0);
       const int64_t prow = (is_main_q ? 0 : a.n_main_pad) + row0;
-      bulk_load(smem_u32(sm.rec[ds]), a.rec + rec_block(rec_kind + h, a.rows_pad, prow), kQc * 16,
-                dbar);
+      bulk_load(smem_u32(sm.rec[ds]), a.rec + rec_block(h, a.rows_pad, prow), kQc * 8, dbar);
       ++do_issued;
     }
     // no copy may still be writing shared memory when the CTA exits
@@ -589,6 +596,10 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const int key = key0 + row;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale_log2;
+    // the query rows that see this key: main rows [x, y), branch rows [z, w)
+    int4 kiv = make_int4(0, 0, 0, 0);
+    if (key < n_keys)
+      kiv = reinterpret_cast<const int4 *>(a.plan.key_iv)[(main_kv ? 0 : a.n_main) + key];
     bool ok = true;
     for (int c = 0; c < total; ++c) {
       const int ds = c % kDoStages;
@@ -610,17 +621,14 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       // this quarter's 32 queries of each record field, four per 16-byte load
       const float4 *r_lse = reinterpret_cast<const float4 *>(sm.rec[ds] + kRecLse + qq * 32);
       const float4 *r_d = reinterpret_cast<const float4 *>(sm.rec[ds] + kRecD + qq * 32);
-      if (!sm.chunk_full[ds]) {
-        const int4 *r_lo = reinterpret_cast<const int4 *>(sm.rec[ds] + kRecLo + qq * 32);
-        const int4 *r_hi = reinterpret_cast<const int4 *>(sm.rec[ds] + kRecHi + qq * 32);
+      const int4 ch = sm.chunk[ds];
+      if (!ch.x) {
+        // queries q of this quarter with lo <= q < hi see the key
+        const int base = ch.z + qq * 32;
+        const int lo = (ch.y ? kiv.z : kiv.x) - base, hi = (ch.y ? kiv.w : kiv.y) - base;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const int4 lo = r_lo[q4], hi = r_hi[q4];
-          if (key < lo.x || key > hi.x) p[4 * q4] = kNegInf;
-          if (key < lo.y || key > hi.y) p[4 * q4 + 1] = kNegInf;
-          if (key < lo.z || key > hi.z) p[4 * q4 + 2] = kNegInf;
-          if (key < lo.w || key > hi.w) p[4 * q4 + 3] = kNegInf;
-        }
+        for (int q = 0; q < 32; ++q)
+          if (q < lo || q >= hi) p[q] = kNegInf;
       }
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
@@ -744,13 +752,13 @@ ba_status launch_bwd_sm100(const AttnParams &a, cudaStream_t s) {
   const int64_t grid_dq = (int64_t)a.n_qt * a.hq;
   const int64_t grid_kv = (int64_t)(a.n_kt + a.n_bkt) * a.hkv;
   if (d == 64) {
-    if ((st = launch_kernel(dkdv_sm100_kernel<64>, sizeof(DkvSmem<64>) + 1024, grid_kv, kDkvThreads, a,
+    if ((st = launch_kernel(dkdv_sm100_kernel<64>, sizeof(DkvSmem<64>), grid_kv, kDkvThreads, a,
                             kvm, s, "dkdv_sm100_kernel<64>")) != BA_OK)
       return st;
     return launch_kernel(dq_sm100_kernel<64>, sizeof(DqSmem<64>) + 1024, grid_dq, kDqThreads, a, dqm, s,
                          "dq_sm100_kernel<64>");
   }
-  if ((st = launch_kernel(dkdv_sm100_kernel<128>, sizeof(DkvSmem<128>) + 1024, grid_kv, kDkvThreads, a,
+  if ((st = launch_kernel(dkdv_sm100_kernel<128>, sizeof(DkvSmem<128>), grid_kv, kDkvThreads, a,
                           kvm, s, "dkdv_sm100_kernel<128>")) != BA_OK)
     return st;
   return launch_kernel(dq_sm100_kernel<128>, sizeof(DqSmem<128>) + 1024, grid_dq, kDqThreads, a, dqm, s,

@@ -46,8 +46,8 @@ struct FusedSmem {
   bf16 q[2][kQc * D];
   bf16 dout[2][kQc * D];
   bf16 ds[128 * kQc];              // dS^T: two boxes [128 keys][64 queries]
-  alignas(16) float rec[4 * kQc];  // LSE log2[128], D[128], key lo[128], key hi[128]
-  int rec_full;                     // every query of the chunk sees every key of the tile
+  alignas(16) float rec[2 * kQc];  // LSE log2 [128], D [128]
+  int4 rec_chunk;                   // {no mask needed, branch query tile, first query row}
   uint64_t bar_kv;
   uint64_t bar_q_full[2], bar_q_empty[2];
   uint64_t bar_do_full[2], bar_do_empty[2];
@@ -123,7 +123,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const uint32_t t_dk = tmem, t_dv = tmem + D, t_sp = tmem + 2 * D, t_qb = tmem + 2 * D + 128;
   // records of this CTA's key kind: main-key intervals or branch-local ones
-  const int64_t rec_kind = main_kv ? 0 : a.hq;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -174,11 +173,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
             a.plan.qtile + (int64_t)(is_main_q ? tile : a.n_qt_main + tile) * 6;
         full = nrows == kQc && kt >= qt[1] && kt < qt[2];
       }
-      sm.rec_full = full ? 1 : 0;
-      mbar_expect_tx(b_rec, kQc * 16);
+      sm.rec_chunk = make_int4(full ? 1 : 0, is_main_q ? 0 : 1, row0, 0);
+      mbar_expect_tx(b_rec, kQc * 8);
       const int64_t prow = (is_main_q ? 0 : a.n_main_pad) + row0;
-      bulk_load(smem_u32(sm.rec), a.rec + rec_block(rec_kind + h, a.rows_pad, prow), kQc * 16,
-                b_rec);
+      bulk_load(smem_u32(sm.rec), a.rec + rec_block(h, a.rows_pad, prow), kQc * 8, b_rec);
       ++rec_issued;
     }
     // no copy may still be writing shared memory when the CTA exits
@@ -294,6 +292,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
     const float sl2 = a.scale_log2;
     constexpr int kDqCols = D / 4;    // dQ columns this thread sums out of QB
     const uint32_t ds_row = smem_u32(sm.ds) + (qq >> 1) * 16384 + row * 128;
+    // the query rows that see this key: main rows [x, y), branch rows [z, w)
+    int4 kiv = make_int4(0, 0, 0, 0);
+    if (key < n_keys)
+      kiv = reinterpret_cast<const int4 *>(a.plan.key_iv)[(main_kv ? 0 : a.n_main) + key];
     bool ok = true;
     // sums dQ(c) (query row `row` of chunk c, columns [qq D/4, (qq+1) D/4)) into
     // the fp32 accumulator
@@ -338,17 +340,14 @@ __global__ void __launch_bounds__(kFThreads, 1)
       // this quarter's 32 queries of each record field, four per 16-byte load
       const float4 *r_lse = reinterpret_cast<const float4 *>(sm.rec + kRecLse + qq * 32);
       const float4 *r_d = reinterpret_cast<const float4 *>(sm.rec + kRecD + qq * 32);
-      if (!sm.rec_full) {
-        const int4 *r_lo = reinterpret_cast<const int4 *>(sm.rec + kRecLo + qq * 32);
-        const int4 *r_hi = reinterpret_cast<const int4 *>(sm.rec + kRecHi + qq * 32);
+      const int4 ch = sm.rec_chunk;
+      if (!ch.x) {
+        // queries q of this quarter with lo <= q < hi see the key
+        const int base = ch.z + qq * 32;
+        const int lo = (ch.y ? kiv.z : kiv.x) - base, hi = (ch.y ? kiv.w : kiv.y) - base;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const int4 lo = r_lo[q4], hi = r_hi[q4];
-          if (key < lo.x || key > hi.x) p[4 * q4] = kNegInf;
-          if (key < lo.y || key > hi.y) p[4 * q4 + 1] = kNegInf;
-          if (key < lo.z || key > hi.z) p[4 * q4 + 2] = kNegInf;
-          if (key < lo.w || key > hi.w) p[4 * q4 + 3] = kNegInf;
-        }
+        for (int q = 0; q < 32; ++q)
+          if (q < lo || q >= hi) p[q] = kNegInf;
       }
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {

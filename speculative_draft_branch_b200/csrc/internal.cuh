@@ -27,6 +27,7 @@ struct PlanView {
   int32_t *fwd_cost;
   int32_t *bwd_cost;
   int32_t *zz_tiles;   // [C * n_qt * 4] or null
+  int32_t *key_iv;     // [(N + Nb) * 4]
 };
 
 // Everything an attention kernel needs; device pointers only.
@@ -41,12 +42,10 @@ struct AttnParams {
   __nv_bfloat16 *dk_m, *dv_m, *dk_b, *dv_b;
   __nv_bfloat16 *dq_out_m, *dq_out_b;  // dQ written directly (tcgen05 backward)
   int32_t zero_dq_acc;                  // preprocess clears dq_acc
-  // per-query backward records (tcgen05 backward), 16 B per (kind, q head,
-  // padded row); kind 0 carries the main-key interval, 1 the branch-local
-  // one; main rows at [0, n_main_pad), branch rows after.  Each 128-row block
-  // of a (kind, head) is 512 words holding four arrays of 128:
-  // LSE * log2(e), D, key lo, key hi (rec_block below), so one 16-byte load
-  // gives one field of four consecutive queries.
+  // per-query backward records (tcgen05 backward), 8 B per (q head, padded
+  // row); main rows at [0, n_main_pad), branch rows after.  Each 128-row
+  // block of a head is 256 words: LSE * log2(e) [128], then D [128]
+  // (rec_block below), so one 16-byte load gives four consecutive queries.
   float *rec;
   int32_t n_main_pad, rows_pad;
   // zigzag partial output (fp32 O accumulator [(N+Nb), Hq, d], LSE [Hq, N+Nb])
@@ -98,11 +97,11 @@ ba_status launch_exp2_check(const float *x, float *y_fma, float *y_mufu, int64_t
 
 __host__ __device__ inline int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// First word of the 128-row record block holding padded row pr of (kind,
-// head) kh; field f of that row is at + 128 f + (pr % 128).
-constexpr int kRecLse = 0, kRecD = 128, kRecLo = 256, kRecHi = 384;
-__host__ __device__ inline int64_t rec_block(int64_t kh, int32_t rows_pad, int64_t pr) {
-  return (kh * rows_pad + (pr & ~(int64_t)127)) * 4;
+// First word of the 128-row record block holding padded row pr of q head h;
+// field f of that row is at + f + (pr % 128).
+constexpr int kRecLse = 0, kRecD = 128;
+__host__ __device__ inline int64_t rec_block(int64_t h, int32_t rows_pad, int64_t pr) {
+  return (h * rows_pad + (pr & ~(int64_t)127)) * 2;
 }
 
 }  // namespace ba

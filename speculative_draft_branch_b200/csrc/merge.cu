@@ -99,8 +99,7 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int64_t rows, int heads,
 // ---- backward preprocess ---------------------------------------------------
 // D[h, row] = sum_d dO[row, h, d] * O[row, h, d] (fp32 accumulate), rows =
 // main rows then branch rows, and the per-query records the backward reads
-// {l log2 e, D, key lo, key hi} (main-key interval and branch-local interval),
-// laid out as four arrays of 128 per 128-row block.
+// {l log2 e, D}, laid out as two arrays of 128 per 128-row block.
 // A warp takes 32 consecutive rows of one head, one lane per row: each lane
 // streams its row's 2 d bf16 of O and dO (16-byte loads, all issued before
 // the products), and the warp's writes of D and of each record field are
@@ -148,17 +147,15 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(AttnParams a) {
     const_cast<float *>(a.d_all)[(int64_t)h * rows + row] = s;
     const float l2 = (is_main ? a.lse_m : a.lse_b)[(int64_t)h * (is_main ? a.n_main : a.n_bt) + r] *
                      1.4426950408889634f;
-    const int4 iv = reinterpret_cast<const int4 *>(a.plan.row_iv)[row];
     const int64_t pr = (is_main ? 0 : a.n_main_pad) + r;
     float *r0 = a.rec + rec_block(h, a.rows_pad, pr) + (pr & 127);
-    float *r1 = a.rec + rec_block((int64_t)a.hq + h, a.rows_pad, pr) + (pr & 127);
-    r0[kRecLse] = l2; r0[kRecD] = s; r0[kRecLo] = __int_as_float(iv.x); r0[kRecHi] = __int_as_float(iv.y);
-    r1[kRecLse] = l2; r1[kRecD] = s; r1[kRecLo] = __int_as_float(iv.z); r1[kRecHi] = __int_as_float(iv.w);
+    r0[kRecLse] = l2;
+    r0[kRecD] = s;
   }
-  // padding rows of the records: empty key intervals
+  // padding rows of the records (no query sees a key through them)
   const int pad_m = a.n_main_pad - a.n_main;
   const int pad_b = a.rows_pad - a.n_main_pad - a.n_bt;
-  const int64_t n_pad = (int64_t)(pad_m + pad_b) * a.hq * 2;
+  const int64_t n_pad = (int64_t)(pad_m + pad_b) * a.hq;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_pad;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int per = pad_m + pad_b;
@@ -166,7 +163,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(AttnParams a) {
     const int j = (int)(i % per);
     const int64_t pr = j < pad_m ? a.n_main + j : a.n_main_pad + a.n_bt + (j - pad_m);
     float *rp = a.rec + rec_block(kh, a.rows_pad, pr) + (pr & 127);
-    rp[kRecLse] = 0.f; rp[kRecD] = 0.f; rp[kRecLo] = __int_as_float(1); rp[kRecHi] = __int_as_float(0);
+    rp[kRecLse] = 0.f;
+    rp[kRecD] = 0.f;
   }
 }
 

@@ -115,6 +115,42 @@ __global__ void plan_rows_kernel(const int32_t *cu, const int32_t *anchor, int n
   }
 }
 
+// ---- per key row: the query rows that see it ------------------------------
+// Query rows of one kind (main rows, branch rows) have non-decreasing lower
+// and upper key bounds (packed order; anchors non-decreasing), so the rows
+// that see key k are one range: from the first row whose upper bound reaches
+// k to the first row whose lower bound passes it.
+__device__ int first_row_at_least(const int32_t *row_iv, int base, int n, int field, int k) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (row_iv[(int64_t)(base + mid) * 4 + field] >= k) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
+__device__ int2 rows_seeing(const int32_t *row_iv, int base, int n, int f_lo, int f_hi, int k) {
+  const int b = first_row_at_least(row_iv, base, n, f_hi, k);
+  const int e = first_row_at_least(row_iv, base, n, f_lo, k + 1);
+  return b < e ? make_int2(b, e) : make_int2(0, 0);
+}
+
+__global__ void plan_key_iv_kernel(int n_main, int n_bt, const int32_t *status,
+                                   const int32_t *row_iv, int32_t *key_iv) {
+  if (status[0] != 0) return;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)n_main + n_bt) return;
+  int2 m = make_int2(0, 0), b;
+  if (i < n_main) {
+    m = rows_seeing(row_iv, 0, n_main, 0, 1, (int)i);
+    b = rows_seeing(row_iv, n_main, n_bt, 0, 1, (int)i);
+  } else {
+    b = rows_seeing(row_iv, n_main, n_bt, 2, 3, (int)(i - n_main));
+  }
+  reinterpret_cast<int4 *>(key_iv)[i] = make_int4(m.x, m.y, b.x, b.y);
+}
+
 // ---- K3: per query tile key ranges ----------------------------------------
 __global__ void plan_tiles_kernel(int n_main, int n_bt, int n_br, int n_qt_main, int n_qt,
                                   const int32_t *status, const int32_t *cu_branch,
@@ -403,7 +439,10 @@ ba_status launch_plan(const ba_problem &p, const ba_plan_layout &L, const PlanVi
       v.status, v.fwd_cost, n_qt, v.fwd_order);
   plan_rank_kernel<<<(unsigned)cdiv64(n_kv, kRankThreads), kRankThreads, 0, s>>>(
       v.status, v.bwd_cost, n_kv, v.bwd_order);
-  count_launches(6);
+  const int64_t n_keys = (int64_t)p.n_main + p.n_branch_tokens;
+  plan_key_iv_kernel<<<(unsigned)cdiv64(n_keys, 256), 256, 0, s>>>(
+      p.n_main, p.n_branch_tokens, v.status, v.row_iv, v.key_iv);
+  count_launches(7);
   if (p.zigzag_C > 1) {
     count_launches(1);
     const int64_t n = (int64_t)p.zigzag_C * n_qt;

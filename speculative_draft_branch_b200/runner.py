@@ -87,6 +87,7 @@ class BranchAttention:
             "kv_branch": arr(L["off_kv_branch"], L["n_kv_branch"], 2),
             "fwd_order": arr(L["off_fwd_order"], n_qt),
             "bwd_order": arr(L["off_bwd_order"], n_kv),
+            "key_iv": arr(L["off_key_iv"], rows, 4),
         }
         if c.zigzag_C > 1:
             out["zz_tiles"] = arr(L["off_zz_tiles"], c.zigzag_C * n_qt, 4).reshape(

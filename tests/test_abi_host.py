@@ -75,8 +75,8 @@ def test_workspace_sizes_follow_the_layout():
     assert fwd_b == 0
     rows = 256 + 768
     rows_pad = 256 + 768          # both kinds already multiples of 128
-    # D [Hq, rows], records 2 x [Hq, rows_pad] float4, fp32 dQ accumulator
-    assert bwd_b == 4 * rows * 4 + 2 * 16 * rows_pad * 4 + 4 * rows * 4 * 64
+    # D [Hq, rows], records [Hq, rows_pad] x {LSE, D} fp32, fp32 dQ accumulator
+    assert bwd_b == 4 * rows * 4 + 8 * rows_pad * 4 + 4 * rows * 4 * 64
     # arrays are 256-byte aligned and do not overlap
     offs = sorted(getattr(L, f) for f, _ in ba.BAPlanLayout._fields_ if f.startswith("off_"))
     assert all(o % 256 == 0 for o in offs)

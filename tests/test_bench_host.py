@@ -75,9 +75,9 @@ def test_hbm_steps_byte_accounting(monkeypatch):
         assert m["ms"] == pytest.approx(0.1)          # 10 calls between two ticks
         p = res["bwd_preprocess"]
         assert p["ms"] == pytest.approx(2.0)
-        # O, dO, LSE read, D and two records written per row-head (plus the zeroed
-        # fp32 dQ accumulator of the fused backward), key interval read per row
-        assert p["bytes_per_launch"] == 4000 * 4 * (2 * 64 * 2 + 4 + 4 + 32 + zero) + 4000 * 16
+        # O, dO, LSE read, D and the {LSE, D} record written per row-head (plus
+        # the zeroed fp32 dQ accumulator of the fused backward)
+        assert p["bytes_per_launch"] == 4000 * 4 * (2 * 64 * 2 + 4 + 4 + 8 + zero)
         assert p["frac"] == pytest.approx(p["achieved"] / 1000.0)
         assert p["achieved"] == pytest.approx(p["bytes_per_launch"] / 2e-3 / 1e9)
 
