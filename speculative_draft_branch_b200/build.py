@@ -3,8 +3,8 @@
     python speculative_draft_branch_b200/build.py [--force] [--verbose]
 
 Every .cu file under csrc/ is compiled separately (parallel) and linked into
-one shared library next to this file.  Rebuilds only what changed, judged
-by a content hash of each output's sources, headers and command line.
+one shared library next to this file.  Rebuilds only what changed, as
+decided by a content hash of each output's sources, headers and command line.
 """
 from __future__ import annotations
 
