@@ -118,7 +118,10 @@ typedef struct {
 /* Byte offsets of the metadata arrays inside a plan workspace (all int32).
  * Query tiles are BA_TILE_M rows (main tiles first, then branch tiles), key
  * tiles BA_TILE_N rows.
- *   status      [4]           word 0 = OR of BA_META_* bits
+ *   status      [4]           word 0 = OR of BA_META_* bits; word 1 = sites of
+ *               bounded device waits that gave up; word 2 = the backward's
+ *               whole walk, the sum over key tiles of the query tiles visiting
+ *               them (sets the backward's launch order)
  *   cu_branch   [n_branches+1]  exclusive scan of branch_depth
  *   branch_seq  [n_branches]    sequence holding each anchor
  *   row_iv      [(n_main + n_branch_tokens) * 4]  per query row: first and

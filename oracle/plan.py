@@ -25,7 +25,8 @@ this library's contract, written in the plain per-tile form:
   * per branch key tile k' (rows [k' BN, (k'+1) BN)): the branch query tiles
     whose branch-local range meets it;
   * forward / backward work orders: tiles sorted by decreasing cost, ties by
-    index (cost = key tiles visited, query tiles visited);
+    index (cost = key tiles visited, query tiles visited); the backward's
+    whole walk is the sum of the backward costs;
   * zigzag (C > 1): per ring step s and query tile, the key tiles spanned by
     the rows' keys inside chunk j and inside chunk 2C-1-j of their sequence,
     j = (shard(row) - s) mod C, as two ranges (empty = [0, 0)).
@@ -166,6 +167,8 @@ def plan(st, BM: int = PLAN_BM, BN: int = PLAN_BN) -> dict:
         "kv_branch": kv_branch,
         "fwd_order": fwd_order.astype(np.int64),
         "bwd_order": bwd_order.astype(np.int64),
+        # the backward's whole walk: query tiles over all key tiles
+        "walk": int(bwd_cost.sum()),
     }
     C = int(getattr(st, "zigzag_C", 1))
     if C > 1:

@@ -200,10 +200,11 @@ __device__ __forceinline__ int first_greater(const int32_t *qtile, int lo, int h
 
 // ---- K4: per key tile query-tile ranges (backward) -------------------------
 __global__ void plan_kv_kernel(int n_bt, int n_qt_main, int n_qt, int n_kt, int n_bkt,
-                               const int32_t *status, const int32_t *qtile, int32_t *kv_main,
+                               int32_t *status, const int32_t *qtile, int32_t *kv_main,
                                int32_t *kv_branch, int32_t *bwd_cost) {
   if (status[0] != 0) return;
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  int cost = 0;
   if (k < n_kt) {
     int out[4];
 #pragma unroll
@@ -216,7 +217,8 @@ __global__ void plan_kv_kernel(int n_bt, int n_qt_main, int n_qt, int n_kt, int 
     }
     int32_t *o = kv_main + (int64_t)k * 4;
     o[0] = out[0]; o[1] = out[1]; o[2] = out[2]; o[3] = out[3];
-    bwd_cost[k] = (out[1] - out[0]) + (out[3] - out[2]);
+    cost = (out[1] - out[0]) + (out[3] - out[2]);
+    bwd_cost[k] = cost;
   } else if (k < n_kt + n_bkt) {
     const int kb = k - n_kt;
     const int key_lo = kb * kTileN, key_hi = min(key_lo + kTileN, n_bt);
@@ -226,8 +228,12 @@ __global__ void plan_kv_kernel(int n_bt, int n_qt_main, int n_qt, int n_kt, int 
     if (t1 <= t2) { b = t1 - n_qt_main; e = t2 + 1 - n_qt_main; }
     kv_branch[(int64_t)kb * 2] = b;
     kv_branch[(int64_t)kb * 2 + 1] = e;
-    bwd_cost[k] = e - b;
+    cost = e - b;
+    bwd_cost[k] = cost;
   }
+  // status word 2: the backward's whole walk (query tiles over all key tiles)
+  cost = __reduce_add_sync(0xffffffffu, cost);
+  if ((threadIdx.x & 31) == 0 && cost) atomicAdd(status + 2, cost);
 }
 
 // ---- K5: stable order by decreasing cost (rank by counting) ---------------

@@ -79,6 +79,7 @@ class BranchAttention:
 
         out = {
             "status": int(raw[L["off_status"] // 4]),
+            "walk": int(raw[L["off_status"] // 4 + 2]),
             "cu_branch": arr(L["off_cu_branch"], c.n_branches + 1),
             "branch_seq": arr(L["off_branch_seq"], c.n_branches),
             "row_iv": arr(L["off_row_iv"], rows, 4),

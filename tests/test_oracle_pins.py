@@ -389,6 +389,8 @@ def test_plan_matches_bruteforce(kind, seed, tile):
                           p["kv_main"][:, 1] - p["kv_main"][:, 0] + p["kv_main"][:, 3]
                           - p["kv_main"][:, 2], p["kv_branch"][:, 1] - p["kv_branch"][:, 0]]))):
         order = p[key]
+        if key == "bwd_order":
+            assert p["walk"] == int(cost.sum())
         assert sorted(order.tolist()) == list(range(cost.shape[0]))
         for i in range(len(order) - 1):
             a, b = order[i], order[i + 1]
