@@ -121,7 +121,7 @@ typedef struct {
  *   status      [4]           word 0 = OR of BA_META_* bits; word 1 = sites of
  *               bounded device waits that gave up; word 2 = the backward's
  *               whole walk, the sum over key tiles of the query tiles visiting
- *               them (sets the backward's launch order)
+ *               them (the backward's work in chunks; reported, not read back)
  *   cu_branch   [n_branches+1]  exclusive scan of branch_depth
  *   branch_seq  [n_branches]    sequence holding each anchor
  *   row_iv      [(n_main + n_branch_tokens) * 4]  per query row: first and

@@ -198,6 +198,12 @@ AttnParams make_params(const ba_problem &p, const ba_plan_layout &L, const void 
   a.zz_C = p.zigzag_C;
   a.ring = 0;
   a.n_keys_m = p.n_main;
+  {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    a.n_sms = sms > 0 ? sms : 148;
+  }
   return a;
 }
 

@@ -386,9 +386,6 @@ static_assert(sizeof(DkvSmem<128>) <= 232448, "dK/dV kernel exceeds 227 KB of sh
 // and the dS work of chunk c runs under dV(c) and S^T(c+1).
 // 576 threads: warp 0 producer, warp 1 MMA issuer, warps 2-17 P^T / dS^T.
 constexpr int kDkvThreads = 576;
-// walk (plan status word 2) from which the kv group goes outermost: between
-// the 64K DSpark-style batch (1.6e5) and the 256K TTT sequence (8.4e6)
-constexpr int kGroupOuterWalk = 1 << 20;
 constexpr int kDkvElem = kDkvThreads - 64;   // P^T / dS^T threads
 
 template <int D>
@@ -406,17 +403,18 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   }
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // Launch order.  A backward with a long walk runs for seconds under the
-  // power cap, where DRAM traffic costs clock: the kv group then goes
-  // outermost, so the CTAs resident at one time walk the same q heads' query
-  // tiles and share their Q / dO tiles in L2 (about a quarter of the DRAM
-  // reads).  Shorter backwards keep the kv groups of one key tile side by
-  // side, which measured faster without the cap.
+  // Launch order: the plan's longest-first key tiles in bands of one CTA per
+  // SM, each band run kv group by kv group.  A wave is then one kv group's
+  // adjacent key tiles, which walk the same q heads' query tiles and share
+  // their Q / dO tiles in L2, and the longest walks still start first.
   const int n_items = a.n_kt + a.n_bkt;
-  const bool group_outer = a.plan.status[2] >= kGroupOuterWalk;
-  const int item =
-      a.plan.bwd_order[group_outer ? (int)(blockIdx.x % n_items) : (int)(blockIdx.x / a.hkv)];
-  const int g = group_outer ? (int)(blockIdx.x / n_items) : (int)(blockIdx.x % a.hkv);
+  const int band = a.n_sms;
+  const int per_band = band * a.hkv;
+  const int b0 = (int)(blockIdx.x / per_band) * band;       // first item of this band
+  const int width = min(band, n_items - b0);                  // items in this band
+  const int in_band = (int)(blockIdx.x % per_band);
+  const int g = in_band / width;
+  const int item = a.plan.bwd_order[b0 + in_band % width];
   const bool main_kv = item < a.n_kt;
   const int kt = main_kv ? item : item - a.n_kt;
   const int key0 = kt * 128;

@@ -58,6 +58,7 @@ struct AttnParams {
   // step C takes the branch-local keys (row_iv z, w; qtile[4..5])
   int32_t ring;
   int32_t n_keys_m;           // main key rows (the visiting shard's in ring mode, else n_main)
+  int32_t n_sms;              // streaming multiprocessors of the device (launch-order bands)
   const int32_t *cu_seqlens;
   PlanView plan;
   int32_t n_main, n_bt;       // main / branch token counts
