@@ -142,14 +142,17 @@ typedef struct {
  *               first): the main query rows that see it [x, y) and the branch
  *               query rows that see it [z, w) (branch rows counted from 0);
  *               empty = (0, 0).  Contiguous because row bounds are
- *               non-decreasing; used by the backward's key-stationary walk. */
+ *               non-decreasing; used by the backward's key-stationary walk.
+ *   bwd_prefix  [n_kv_main + n_kv_branch]  walk ahead of each position of
+ *               bwd_order: the sum of bwd_cost over the key tiles ranked
+ *               before it (the dK/dV launch order reads it). */
 #define BA_TILE_M 128
 #define BA_TILE_N 128
 typedef struct {
   size_t total_bytes;
   size_t off_status, off_cu_branch, off_branch_seq, off_row_iv, off_qtile;
   size_t off_kv_main, off_kv_branch, off_fwd_order, off_bwd_order;
-  size_t off_fwd_cost, off_bwd_cost, off_zz_tiles, off_key_iv;
+  size_t off_fwd_cost, off_bwd_cost, off_zz_tiles, off_key_iv, off_bwd_prefix;
   int32_t n_qtiles_main, n_qtiles_branch, n_kv_main, n_kv_branch;
 } ba_plan_layout;
 

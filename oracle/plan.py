@@ -169,6 +169,8 @@ def plan(st, BM: int = PLAN_BM, BN: int = PLAN_BN) -> dict:
         "bwd_order": bwd_order.astype(np.int64),
         # the backward's whole walk: query tiles over all key tiles
         "walk": int(bwd_cost.sum()),
+        # walk ahead of each position of the backward order
+        "bwd_prefix": (np.cumsum(bwd_cost[bwd_order]) - bwd_cost[bwd_order]).astype(np.int64),
     }
     C = int(getattr(st, "zigzag_C", 1))
     if C > 1:

@@ -52,7 +52,7 @@ class BAPlanLayout(ctypes.Structure):
         (name, ctypes.c_size_t) for name in (
             "off_status", "off_cu_branch", "off_branch_seq", "off_row_iv", "off_qtile",
             "off_kv_main", "off_kv_branch", "off_fwd_order", "off_bwd_order", "off_fwd_cost",
-            "off_bwd_cost", "off_zz_tiles", "off_key_iv")] + [
+            "off_bwd_cost", "off_zz_tiles", "off_key_iv", "off_bwd_prefix")] + [
         (name, ctypes.c_int32) for name in (
             "n_qtiles_main", "n_qtiles_branch", "n_kv_main", "n_kv_branch")]
 

@@ -131,6 +131,7 @@ void plan_layout(const ba_problem &p, ba_plan_layout *L) {
   L->off_bwd_cost = take(4 * (size_t)n_kv);
   L->off_zz_tiles = take(p.zigzag_C > 1 ? 16 * (size_t)p.zigzag_C * n_qt : 0);
   L->off_key_iv = take(16 * (size_t)rows);
+  L->off_bwd_prefix = take(4 * (size_t)n_kv);
   L->total_bytes = off;
 }
 
@@ -150,6 +151,7 @@ PlanView plan_view(const ba_plan_layout &L, const void *ws) {
   v.bwd_cost = reinterpret_cast<int32_t *>(b + L.off_bwd_cost);
   v.zz_tiles = reinterpret_cast<int32_t *>(b + L.off_zz_tiles);
   v.key_iv = reinterpret_cast<int32_t *>(b + L.off_key_iv);
+  v.bwd_prefix = reinterpret_cast<int32_t *>(b + L.off_bwd_prefix);
   return v;
 }
 

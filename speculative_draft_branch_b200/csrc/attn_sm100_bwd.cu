@@ -404,17 +404,29 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // Launch order: the plan's longest-first key tiles in bands of one CTA per
-  // SM, each band run kv group by kv group.  A wave is then one kv group's
-  // adjacent key tiles, which walk the same q heads' query tiles and share
-  // their Q / dO tiles in L2, and the longest walks still start first.
+  // SM.  A band runs kv group by kv group, so that a wave is one kv group's
+  // key tiles, which walk the same q heads' query tiles and share their Q /
+  // dO tiles in L2.  That starts the band's longest walk of the last kv group
+  // after the walk ahead of the band and (hkv-1)/hkv of the band's own, spread
+  // over the SMs; where it would then end more than a quarter past the
+  // launch's balanced end (hkv * walk / n_sms), the band keeps the kv groups
+  // of a key tile side by side instead, longest walks first.
   const int n_items = a.n_kt + a.n_bkt;
   const int band = a.n_sms;
   const int per_band = band * a.hkv;
   const int b0 = (int)(blockIdx.x / per_band) * band;       // first item of this band
   const int width = min(band, n_items - b0);                  // items in this band
   const int in_band = (int)(blockIdx.x % per_band);
-  const int g = in_band / width;
-  const int item = a.plan.bwd_order[b0 + in_band % width];
+  const int64_t walk = a.plan.status[2];
+  const int64_t ahead = a.plan.bwd_prefix[b0];
+  const int64_t next = b0 + 1 < n_items ? a.plan.bwd_prefix[b0 + 1] : walk;
+  const int64_t end = b0 + width < n_items ? a.plan.bwd_prefix[b0 + width] : walk;
+  const int item_g = a.plan.bwd_order[b0 + in_band % width];
+  const int item_k = a.plan.bwd_order[b0 + in_band / a.hkv];
+  const int64_t finish = a.hkv * ahead + (a.hkv - 1) * (end - ahead) + (int64_t)a.n_sms * (next - ahead);
+  const bool by_group = 4 * finish <= 5 * (int64_t)a.hkv * walk;
+  const int g = by_group ? in_band / width : in_band % a.hkv;
+  const int item = by_group ? item_g : item_k;
   const bool main_kv = item < a.n_kt;
   const int kt = main_kv ? item : item - a.n_kt;
   const int key0 = kt * 128;

@@ -28,6 +28,7 @@ struct PlanView {
   int32_t *bwd_cost;
   int32_t *zz_tiles;   // [C * n_qt * 4] or null
   int32_t *key_iv;     // [(N + Nb) * 4]
+  int32_t *bwd_prefix; // [n_kt + n_bkt] bwd_cost summed over the key tiles ranked before
 };
 
 // Everything an attention kernel needs; device pointers only.

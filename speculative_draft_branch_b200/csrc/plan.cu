@@ -237,15 +237,17 @@ __global__ void plan_kv_kernel(int n_bt, int n_qt_main, int n_qt, int n_kt, int 
 }
 
 // ---- K5: stable order by decreasing cost (rank by counting) ---------------
+// prefix (optional): at each position of the order, the cost summed over the
+// entries ranked before it.
 constexpr int kRankThreads = 256;
 __global__ void __launch_bounds__(kRankThreads) plan_rank_kernel(const int32_t *status,
                                                                  const int32_t *cost, int n,
-                                                                 int32_t *order) {
+                                                                 int32_t *order, int32_t *prefix) {
   if (status[0] != 0) return;
   __shared__ int32_t sc[kRankThreads];
   const int i = blockIdx.x * kRankThreads + threadIdx.x;
   const int ci = i < n ? cost[i] : 0;
-  int rank = 0;
+  int rank = 0, ahead = 0;
   for (int base = 0; base < n; base += kRankThreads) {
     __syncthreads();
     int j = base + threadIdx.x;
@@ -255,10 +257,15 @@ __global__ void __launch_bounds__(kRankThreads) plan_rank_kernel(const int32_t *
     for (int u = 0; u < lim; ++u) {
       int cu_ = sc[u];
       int j2 = base + u;
-      rank += (cu_ > ci) || (cu_ == ci && j2 < i);
+      const bool before = (cu_ > ci) || (cu_ == ci && j2 < i);
+      rank += before;
+      ahead += before ? cu_ : 0;
     }
   }
-  if (i < n) order[rank] = i;
+  if (i < n) {
+    order[rank] = i;
+    if (prefix) prefix[rank] = ahead;
+  }
 }
 
 // ---- K6: zigzag ring-step key-tile ranges ----------------------------------
@@ -417,7 +424,7 @@ ba_status launch_ring_plan(const ba_problem &p, const ba_plan_layout &L, const P
       p.n_main, p.n_branch_tokens, L.n_qtiles_main, n_qt, v.status, v.row_iv, v.qtile,
       v.fwd_cost);
   plan_rank_kernel<<<(unsigned)cdiv64(n_qt, kRankThreads), kRankThreads, 0, s>>>(
-      v.status, v.fwd_cost, n_qt, v.fwd_order);
+      v.status, v.fwd_cost, n_qt, v.fwd_order, nullptr);
   count_launches(4);
   return cuda_check(cudaGetLastError(), "ring plan kernels launch");
 }
@@ -442,9 +449,9 @@ ba_status launch_plan(const ba_problem &p, const ba_plan_layout &L, const PlanVi
       p.n_branch_tokens, L.n_qtiles_main, n_qt, L.n_kv_main, L.n_kv_branch, v.status,
       v.qtile, v.kv_main, v.kv_branch, v.bwd_cost);
   plan_rank_kernel<<<(unsigned)cdiv64(n_qt, kRankThreads), kRankThreads, 0, s>>>(
-      v.status, v.fwd_cost, n_qt, v.fwd_order);
+      v.status, v.fwd_cost, n_qt, v.fwd_order, nullptr);
   plan_rank_kernel<<<(unsigned)cdiv64(n_kv, kRankThreads), kRankThreads, 0, s>>>(
-      v.status, v.bwd_cost, n_kv, v.bwd_order);
+      v.status, v.bwd_cost, n_kv, v.bwd_order, v.bwd_prefix);
   const int64_t n_keys = (int64_t)p.n_main + p.n_branch_tokens;
   plan_key_iv_kernel<<<(unsigned)cdiv64(n_keys, 256), 256, 0, s>>>(
       p.n_main, p.n_branch_tokens, v.status, v.row_iv, v.key_iv);

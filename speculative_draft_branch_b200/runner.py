@@ -89,6 +89,7 @@ class BranchAttention:
             "fwd_order": arr(L["off_fwd_order"], n_qt),
             "bwd_order": arr(L["off_bwd_order"], n_kv),
             "key_iv": arr(L["off_key_iv"], rows, 4),
+            "bwd_prefix": arr(L["off_bwd_prefix"], n_kv),
         }
         if c.zigzag_C > 1:
             out["zz_tiles"] = arr(L["off_zz_tiles"], c.zigzag_C * n_qt, 4).reshape(

@@ -391,6 +391,12 @@ def test_plan_matches_bruteforce(kind, seed, tile):
         order = p[key]
         if key == "bwd_order":
             assert p["walk"] == int(cost.sum())
+            # walk ahead of each position, summed one entry at a time
+            ahead = 0
+            for i, k in enumerate(order):
+                assert p["bwd_prefix"][i] == ahead
+                ahead += int(cost[k])
+            assert ahead == p["walk"]
         assert sorted(order.tolist()) == list(range(cost.shape[0]))
         for i in range(len(order) - 1):
             a, b = order[i], order[i + 1]
