@@ -691,9 +691,9 @@ __global__ void __launch_bounds__(384, 1)
       }
       float mx4[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
 #pragma unroll
-      for (int c = 0; c < 128; c += 4) {
+      for (int c = 0; c < 128; c += 8) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) mx4[e] = fmaxf(mx4[e], s[c + e]);
+        for (int e = 0; e < 4; ++e) mx4[e] = fmax3(mx4[e], s[c + e], s[c + 4 + e]);
       }
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
       const float m_new = fmaxf(m_used, mx);
@@ -719,20 +719,26 @@ __global__ void __launch_bounds__(384, 1)
       // P = 2^(s sl2 - m), packed to bf16 pairs in place, written over the
       // first 64 columns of this head's S (all of S is in registers now)
       uint32_t *pk = reinterpret_cast<uint32_t *>(s);
-      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      // scale and shift, and the row sums, on fp32 pairs
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm = f2_pack(-msub, -msub);
+      uint64_t l01 = f2_pack(0.f, 0.f), l23 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 128; c += 4) {
-        float pv[4];
+        float pv[4], x[4];
+        f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm), x[0], x[1]);
+        f2_unpack(f2_fma(f2_pack(s[c + 2], s[c + 3]), sl2x2, negm), x[2], x[3]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          pv[e] = ex2(fmaf(s[c + e], sl2, -msub));
-          l4[e] += pv[e];
-        }
+        for (int e = 0; e < 4; ++e) pv[e] = ex2(x[e]);
+        l01 = f2_add(l01, f2_pack(pv[0], pv[1]));
+        l23 = f2_add(l23, f2_pack(pv[2], pv[3]));
         pk[c / 2] = pack_bf16(pv[0], pv[1]);
         pk[c / 2 + 1] = pack_bf16(pv[2], pv[3]);
       }
       tmem_st32(ts, pk);
       tmem_st32(ts + 32, pk + 32);
+      float l4[4];
+      f2_unpack(l01, l4[0], l4[1]);
+      f2_unpack(l23, l4[2], l4[3]);
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       tc_wait_st();
       tc_fence_before();

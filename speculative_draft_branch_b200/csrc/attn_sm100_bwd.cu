@@ -281,16 +281,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
       }
       const float sl2 = a.scale_log2;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), nl2 = f2_pack(-lse2, -lse2), dd2 = f2_pack(dd, dd);
       uint32_t *pk = reinterpret_cast<uint32_t *>(dp);
 #pragma unroll
       for (int c = 0; c < 32; c += 2) {
-        float d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float p = ex2(fmaf(s[c + e], sl2, -lse2));
-          d2[e] = p * (dp[c + e] - dd);
-        }
-        pk[c / 2] = pack_bf16(d2[0], d2[1]);
+        float x0, x1, d0, d1;
+        f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, nl2), x0, x1);
+        f2_unpack(f2_mul(f2_pack(ex2(x0), ex2(x1)), f2_sub(f2_pack(dp[c], dp[c + 1]), dd2)), d0, d1);
+        pk[c / 2] = pack_bf16(d0, d1);
       }
       // dS buffer j&1 was last read by dQ_{j-2}
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.bar_dq_done[j & 1]),
@@ -680,9 +678,15 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
         const float4 dd = r_d[q4];
-        dk2[2 * q4] = pack_bf16(p[4 * q4] * (dp[4 * q4] - dd.x), p[4 * q4 + 1] * (dp[4 * q4 + 1] - dd.y));
-        dk2[2 * q4 + 1] =
-            pack_bf16(p[4 * q4 + 2] * (dp[4 * q4 + 2] - dd.z), p[4 * q4 + 3] * (dp[4 * q4 + 3] - dd.w));
+        float d[4];
+        f2_unpack(f2_mul(f2_pack(p[4 * q4], p[4 * q4 + 1]),
+                         f2_sub(f2_pack(dp[4 * q4], dp[4 * q4 + 1]), f2_pack(dd.x, dd.y))),
+                  d[0], d[1]);
+        f2_unpack(f2_mul(f2_pack(p[4 * q4 + 2], p[4 * q4 + 3]),
+                         f2_sub(f2_pack(dp[4 * q4 + 2], dp[4 * q4 + 3]), f2_pack(dd.z, dd.w))),
+                  d[2], d[3]);
+        dk2[2 * q4] = pack_bf16(d[0], d[1]);
+        dk2[2 * q4 + 1] = pack_bf16(d[2], d[3]);
       }
       tmem_st16(coly, dk2);
       tc_wait_st();
